@@ -1,0 +1,391 @@
+"""Plain CPU oracle for the LoopKV decode path.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+CPU-baseline / reference legs of the benchmark may import this module.  The
+product path (the CUDA library and its Python binding) never calls it and
+shares no code with it.
+
+What it computes, following LoopKV: Loop-Aware KV Cache Compression for
+Serving Looped Transformers (Abstract):
+  * every (loop, layer) cell is stored 4-bit, 2-bit, or reuses the final
+    loop's cell of the same layer;
+  * a 4-bit code is kept as a high-2-bit plane and a low-2-bit plane; during
+    decoding the high plane of every value is read and the low plane only for
+    tokens whose own attention weight needs full precision.
+
+The pages leave the quantiser and the threshold rule open; this oracle takes
+the readings the library documents:
+  * asymmetric b-bit quantisation, keys per channel over 32-token groups
+    aligned at positions 0, 32, 64, ..., values per token over 32-channel
+    groups; scale and minimum rounded to bf16 (round to nearest even);
+  * quantiser arithmetic in fp32, one correctly rounded operation at a time,
+    because its result is an integer code that both sides must agree on;
+  * key tokens of an unfinished group stay exact (bf16) until the group fills;
+  * a value's high-plane-only reconstruction is the bucket midpoint
+    ``min + scale * (4 * hi + 1.5)``;
+  * a token takes the low plane when its softmax weight, rounded to fp32, is
+    at least tau (tau = 0 selects every token, tau = +inf none);
+  * attention itself is evaluated in fp64.
+
+Byte layout (the oracle's own reading of the record format, used only to
+compare the library's packed bytes): per (physical block, head) record of
+``block_size`` (16) tokens,
+  4-bit: [K hi plane][K lo plane][K meta][V hi plane][V meta][V lo plane]
+  2-bit: [K plane][K meta][V plane][V meta]
+  bf16 : [K rows][V rows]
+A plane row is one token, channel c at byte c // 4, bits 2 * (c % 4) and up.
+K meta holds (scale, min) bf16 pairs of half the channels of the 32-token
+group: channels [0, D/2) in the group's even block, [D/2, D) in the odd one.
+V meta holds (scale, min) per token row and 32-channel group.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+GROUP = 32          # quantisation group (tokens for keys, channels for values)
+BLOCK = 16          # tokens per paged block
+
+BITS = {"q4": 4, "q2": 2}
+
+
+# ---------------------------------------------------------------------------
+# bf16 helpers
+# ---------------------------------------------------------------------------
+
+def bf16_round(x) -> np.ndarray:
+    """Round fp32 values to the nearest bf16 (ties to even); returns fp32."""
+    x = np.asarray(x, dtype=np.float32)
+    shape = x.shape
+    u = np.ascontiguousarray(x).reshape(-1).view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    r = ((u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)) << np.uint64(16)
+    return r.astype(np.uint32).view(np.float32).reshape(shape)
+
+
+def bf16_bits(x) -> np.ndarray:
+    """uint16 bit patterns of bf16-exact fp32 values."""
+    x = np.asarray(x, dtype=np.float32)
+    u = np.ascontiguousarray(x).reshape(-1).view(np.uint32).reshape(x.shape)
+    if np.any(u & np.uint32(0xFFFF)):
+        raise ValueError("value is not bf16-exact")
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+# ---------------------------------------------------------------------------
+# Quantiser
+# ---------------------------------------------------------------------------
+
+def quantize_group(x, bits: int):
+    """Asymmetric ``bits``-bit quantisation of the last axis (one group).
+
+    Returns (codes uint8[..., G], scale fp32[...], minimum fp32[...]); scale
+    and minimum are bf16-exact.  Steps, each a single fp32 operation:
+      mn_b = bf16(min x);  s_b = bf16((max x - mn_b) / (2^b - 1));
+      code = clamp(rint_half_even((x - mn_b) / s_b), 0, 2^b - 1), 0 if s_b = 0.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    levels = np.float32(2 ** bits - 1)
+    mn = x.min(axis=-1)
+    mx = x.max(axis=-1)
+    mn_b = bf16_round(mn)
+    s_b = bf16_round((mx - mn_b) / levels)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (x - mn_b[..., None]) / s_b[..., None]
+    codes = np.where(s_b[..., None] == 0, np.float32(0),
+                     np.clip(np.rint(t), np.float32(0), levels))
+    return codes.astype(np.uint8), s_b.astype(np.float32), mn_b.astype(np.float32)
+
+
+class QuantKeys:
+    """Keys of one (sequence, head): complete 32-token groups quantised per
+    channel, the tail of an unfinished group kept exact."""
+
+    def __init__(self, k: np.ndarray, bits: int):
+        k = np.asarray(k, dtype=np.float32)
+        n, d = k.shape
+        ng = n // GROUP
+        self.bits, self.n, self.d = bits, n, d
+        grouped = k[: ng * GROUP].reshape(ng, GROUP, d).transpose(0, 2, 1)  # [g, ch, tok]
+        codes, s, mn = quantize_group(grouped, bits)
+        self.codes = codes.transpose(0, 2, 1).reshape(ng * GROUP, d)       # [tok, ch]
+        self.scale = s            # [g, ch]
+        self.minv = mn            # [g, ch]
+        self.residual = k[ng * GROUP:].copy()                              # [n % 32, ch]
+
+    def dequant(self) -> np.ndarray:
+        ng = self.codes.shape[0] // GROUP
+        out = np.empty((self.n, self.d), dtype=np.float64)
+        if ng:
+            c = self.codes.reshape(ng, GROUP, self.d).astype(np.float64)
+            s = self.scale.astype(np.float64)[:, None, :]
+            m = self.minv.astype(np.float64)[:, None, :]
+            out[: ng * GROUP] = (m + s * c).reshape(ng * GROUP, self.d)
+        out[ng * GROUP:] = self.residual
+        return out
+
+
+class QuantValues:
+    """Values of one (sequence, head), quantised per token over 32-channel groups."""
+
+    def __init__(self, v: np.ndarray, bits: int):
+        v = np.asarray(v, dtype=np.float32)
+        n, d = v.shape
+        self.bits, self.n, self.d = bits, n, d
+        codes, s, mn = quantize_group(v.reshape(n, d // GROUP, GROUP), bits)
+        self.codes = codes.reshape(n, d)     # [tok, ch]
+        self.scale = s                       # [tok, d/32]
+        self.minv = mn                       # [tok, d/32]
+
+    def _expand(self, a):
+        return np.repeat(a.astype(np.float64), GROUP, axis=1)
+
+    def dequant_full(self) -> np.ndarray:
+        return self._expand(self.minv) + self._expand(self.scale) * self.codes.astype(np.float64)
+
+    def dequant_high(self) -> np.ndarray:
+        """High-plane-only reconstruction of a 4-bit value: bucket midpoint."""
+        if self.bits != 4:
+            raise ValueError("high-plane reconstruction is defined for 4-bit cells")
+        hi = (self.codes >> 2).astype(np.float64)
+        return self._expand(self.minv) + self._expand(self.scale) * (4.0 * hi + 1.5)
+
+
+# ---------------------------------------------------------------------------
+# Attention of one (cell, sequence, head)
+# ---------------------------------------------------------------------------
+
+def softmax_weights(q, k_hat, sm_scale: float):
+    """fp64 logits and softmax weights of one query over n keys."""
+    s = float(sm_scale) * (np.asarray(k_hat, np.float64) @ np.asarray(q, np.float64))
+    m = s.max()
+    e = np.exp(s - m)
+    return s, e / e.sum()
+
+
+def select_low_plane(p, tau: float) -> np.ndarray:
+    """Tokens whose fp32 softmax weight is at least tau."""
+    return np.asarray(p, np.float64).astype(np.float32) >= np.float32(tau)
+
+
+def attend(q, k_hat, v_full, v_high, tau: float, sm_scale: float):
+    """Decode attention of one query.
+
+    ``v_high`` is None for cells without a low plane (2-bit, bf16); then every
+    token uses ``v_full`` and nothing is selected.  Returns (o fp64[D],
+    selected bool[n], p fp64[n]).
+    """
+    k_hat = np.asarray(k_hat, np.float64)
+    n, d = k_hat.shape
+    if n == 0:
+        return np.zeros(d), np.zeros(0, dtype=bool), np.zeros(0)
+    _, p = softmax_weights(q, k_hat, sm_scale)
+    if v_high is None:
+        sel = np.zeros(n, dtype=bool)
+        v_hat = np.asarray(v_full, np.float64)
+    else:
+        sel = select_low_plane(p, tau)
+        v_hat = np.where(sel[:, None], v_full, v_high)
+    return p @ v_hat, sel, p
+
+
+class StoredSequence:
+    """One (stored cell, sequence, head): the quantised (or exact) K and V."""
+
+    def __init__(self, kind: str, k, v):
+        self.kind = kind
+        k = np.asarray(k, dtype=np.float32)
+        v = np.asarray(v, dtype=np.float32)
+        self.n = k.shape[0]
+        if kind == "bf16":
+            self.k_exact, self.v_exact = k.copy(), v.copy()
+        elif kind in BITS:
+            self.qk = QuantKeys(k, BITS[kind])
+            self.qv = QuantValues(v, BITS[kind])
+        else:
+            raise ValueError(kind)
+
+    def attend(self, q, tau: float, sm_scale: float):
+        """Attention of one query over every stored token."""
+        if self.kind == "bf16":
+            return attend(q, self.k_exact, self.v_exact, None, tau, sm_scale)
+        k_hat = self.qk.dequant()
+        v_full = self.qv.dequant_full()
+        v_high = self.qv.dequant_high() if self.kind == "q4" else None
+        return attend(q, k_hat, v_full, v_high, tau, sm_scale)
+
+
+def resolve_source(plan, cell: int, num_layers: int) -> int:
+    """A reuse cell reads the final loop's cell of the same layer."""
+    if plan[cell] != "reuse":
+        return cell
+    num_loops = len(plan) // num_layers
+    src = (num_loops - 1) * num_layers + cell % num_layers
+    if plan[src] == "reuse":
+        raise ValueError("the final loop cannot reuse")
+    return src
+
+
+def decode_cell(plan, num_layers: int, cell: int, stored: dict, q, seq_lens,
+                tau: float, sm_scale: float, pairs=None):
+    """Decode attention of one cell for the (b, h) pairs given.
+
+    ``stored[(src_cell, b, h)]`` is the StoredSequence of a stored cell;
+    ``q`` is fp32[B, H, D]; returns {(b, h): (o, selected, p)}.
+    """
+    src = resolve_source(plan, cell, num_layers)
+    out = {}
+    for (b, h) in pairs:
+        seq = stored[(src, b, h)]
+        if int(seq_lens[b]) != seq.n:
+            raise ValueError("sequence length does not match the stored sequence")
+        out[(b, h)] = seq.attend(np.asarray(q[b, h], np.float32), tau, sm_scale)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Byte layout of a stored cell (the oracle's own reading of the record format)
+# ---------------------------------------------------------------------------
+
+def record_sections(kind: str, d: int, block: int = BLOCK):
+    """[(name, offset, size)] of one (block, head) record."""
+    plane = block * d // 4                 # 2 bits per element
+    kmeta = (d // 2) * 4                   # (scale, min) bf16 for half the channels
+    vmeta = block * (d // GROUP) * 4       # (scale, min) bf16 per token and channel group
+    if kind == "q4":
+        sizes = [("k_hi", plane), ("k_lo", plane), ("k_meta", kmeta),
+                 ("v_hi", plane), ("v_meta", vmeta), ("v_lo", plane)]
+    elif kind == "q2":
+        sizes = [("k", plane), ("k_meta", kmeta), ("v", plane), ("v_meta", vmeta)]
+    elif kind == "bf16":
+        sizes = [("k", block * d * 2), ("v", block * d * 2)]
+    else:
+        raise ValueError(kind)
+    out, off = [], 0
+    for name, size in sizes:
+        out.append((name, off, size))
+        off += size
+    return out
+
+
+def record_bytes(kind: str, d: int, block: int = BLOCK) -> int:
+    name, off, size = record_sections(kind, d, block)[-1]
+    return off + size
+
+
+def pack_plane(codes2) -> np.ndarray:
+    """2-bit codes uint8[rows, D] -> plane bytes uint8[rows, D/4]."""
+    c = np.asarray(codes2, dtype=np.uint8)
+    if np.any(c > 3):
+        raise ValueError("plane codes must be 2-bit")
+    rows, d = c.shape
+    c4 = c.reshape(rows, d // 4, 4).astype(np.uint16)
+    return (c4[..., 0] | (c4[..., 1] << 2) | (c4[..., 2] << 4) | (c4[..., 3] << 6)).astype(np.uint8)
+
+
+def _meta_bytes(scale, minv) -> np.ndarray:
+    """(scale, min) bf16 pairs, little-endian, scale first -> uint8[..., 4]."""
+    s = bf16_bits(scale).astype(np.uint32)
+    m = bf16_bits(minv).astype(np.uint32)
+    word = (s | (m << np.uint32(16))).astype("<u4")
+    return word.view(np.uint8).reshape(word.shape + (4,))
+
+
+def sequence_records(kind: str, k, v, block: int = BLOCK):
+    """Expected records of one (cell, sequence, head) after its first n tokens
+    were appended to a zero-filled arena.
+
+    Returns (records uint8[nblocks, rec], residual fp32[n % 32, D] or None).
+    """
+    k = np.asarray(k, np.float32)
+    v = np.asarray(v, np.float32)
+    n, d = k.shape
+    nblocks = -(-n // block)
+    secs = {name: (off, size) for name, off, size in record_sections(kind, d, block)}
+    rec = np.zeros((nblocks, record_bytes(kind, d, block)), dtype=np.uint8)
+    row = d // 4
+
+    def put(blk, name, r, data):
+        off, _ = secs[name]
+        flat = np.asarray(data, np.uint8).ravel()
+        rec[blk, off + r * flat.size: off + (r + 1) * flat.size] = flat
+
+    if kind == "bf16":
+        kb = bf16_bits(k).view(np.uint8).reshape(n, 2 * d)
+        vb = bf16_bits(v).view(np.uint8).reshape(n, 2 * d)
+        for t in range(n):
+            put(t // block, "k", t % block, kb[t])
+            put(t // block, "v", t % block, vb[t])
+        return rec, None
+
+    bits = BITS[kind]
+    qk, qv = QuantKeys(k, bits), QuantValues(v, bits)
+    # values: every token
+    vmeta = _meta_bytes(qv.scale, qv.minv)          # [n, d/32, 4]
+    if kind == "q4":
+        v_hi, v_lo = pack_plane(qv.codes >> 2), pack_plane(qv.codes & 3)
+    else:
+        v_hi, v_lo = pack_plane(qv.codes), None
+    for t in range(n):
+        blk, r = t // block, t % block
+        put(blk, "v_hi" if kind == "q4" else "v", r, v_hi[t])
+        if v_lo is not None:
+            put(blk, "v_lo", r, v_lo[t])
+        put(blk, "v_meta", r, vmeta[t])
+    # keys: complete groups only
+    ng = n // GROUP
+    if kind == "q4":
+        k_hi, k_lo = pack_plane(qk.codes >> 2), pack_plane(qk.codes & 3)
+    else:
+        k_hi, k_lo = pack_plane(qk.codes), None
+    for t in range(ng * GROUP):
+        blk, r = t // block, t % block
+        put(blk, "k_hi" if kind == "q4" else "k", r, k_hi[t])
+        if k_lo is not None:
+            put(blk, "k_lo", r, k_lo[t])
+    kmeta = _meta_bytes(qk.scale, qk.minv)          # [ng, d, 4]
+    half = d // 2
+    blocks_per_group = GROUP // block
+    for g in range(ng):
+        for part in range(blocks_per_group):
+            chans = slice(part * d // blocks_per_group, (part + 1) * d // blocks_per_group)
+            off, size = secs["k_meta"]
+            data = kmeta[g, chans].ravel()
+            rec[g * blocks_per_group + part, off: off + data.size] = data
+    assert half * 4 == secs["k_meta"][1]
+    return rec, qk.residual
+
+
+def unpack_plane(plane_bytes, d: int) -> np.ndarray:
+    """Inverse of pack_plane (used by tests to read records back)."""
+    b = np.asarray(plane_bytes, np.uint8)
+    rows = b.shape[0]
+    out = np.empty((rows, d), dtype=np.uint8)
+    for i in range(4):
+        out[:, i::4] = (b >> (2 * i)) & 3
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic bytes (what one decode launch must read and write)
+# ---------------------------------------------------------------------------
+
+def decode_bytes(kind: str, d: int, n: int, n_selected: int, block: int = BLOCK) -> int:
+    """Bytes one (cell, sequence, head) decode must move: K and V at the cell's
+    precision (4-bit values: high plane for every token, low plane for the
+    selected ones), the exact key tail, the block-table entries, the query and
+    the output."""
+    q_out = 2 * d * 2 + 4 * (-(-n // block))
+    if n == 0:
+        return q_out
+    if kind == "bf16":
+        return q_out + n * 4 * d
+    ng = n // GROUP
+    full = ng * GROUP
+    plane = d // 4
+    k_meta = ng * d * 4
+    tail = (n - full) * d * 2
+    v_meta = n * (d // GROUP) * 4
+    if kind == "q4":
+        return q_out + full * 2 * plane + k_meta + tail + n * plane + v_meta + n_selected * plane
+    return q_out + full * plane + k_meta + tail + n * plane + v_meta

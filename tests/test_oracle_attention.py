@@ -1,0 +1,223 @@
+"""Pins of the oracle's decode attention and low-plane selection.
+
+The method's special cases reduce to textbook attention, which torch's
+float64 ``scaled_dot_product_attention`` computes independently:
+  * tau = 0: every token takes its full 4-bit value;
+  * tau = +inf: every value is its high-plane midpoint;
+  * 2-bit and bf16 cells: plain attention over the dequantised cache.
+General tau is pinned by the decomposition o = attn(high) + sum over the
+selected tokens of p_t * (full - high), with p from torch's softmax, and by
+the invariants |S| <= 1/tau, S monotone in tau, o inside the value hull.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle as O
+
+
+def _bf16(rng, shape, scale=1.0):
+    x = (rng.standard_normal(shape) * scale).astype(np.float32)
+    return torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+
+
+def _case(seed, n=300, d=128, kind="q4", q_scale=1.0):
+    rng = np.random.default_rng(seed)
+    k = _bf16(rng, (n, d))
+    k[:, rng.choice(d, 4, replace=False)] *= 10.0
+    k = torch.from_numpy(k).to(torch.bfloat16).float().numpy()
+    v = _bf16(rng, (n, d))
+    q = _bf16(rng, (d,), q_scale)
+    return q, k, v, O.StoredSequence(kind, k, v)
+
+
+def _sdpa(q, k, v, sm_scale):
+    t = lambda a: torch.from_numpy(np.asarray(a, np.float64))[None, None]
+    return F.scaled_dot_product_attention(t(q)[:, :, None], t(k), t(v), scale=sm_scale)[0, 0, 0].numpy()
+
+
+def _torch_p(q, k, sm_scale):
+    s = torch.from_numpy(np.asarray(k, np.float64)) @ torch.from_numpy(np.asarray(q, np.float64))
+    return torch.softmax(s * sm_scale, dim=0).numpy()
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tau_zero_is_full_4bit_attention(seed):
+    q, k, v, seq = _case(seed, q_scale=2.0)
+    o, sel, _ = seq.attend(q, 0.0, 1.0)
+    assert sel.all()
+    ref = _sdpa(q, seq.qk.dequant(), seq.qv.dequant_full(), 1.0)
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tau_inf_is_high_plane_attention(seed):
+    q, k, v, seq = _case(seed, q_scale=2.0)
+    o, sel, _ = seq.attend(q, math.inf, 1.0)
+    assert not sel.any()
+    ref = _sdpa(q, seq.qk.dequant(), seq.qv.dequant_high(), 1.0)
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", ["q2", "bf16"])
+def test_q2_and_bf16_are_plain_attention(kind):
+    q, k, v, seq = _case(3, kind=kind, q_scale=0.5)
+    o, sel, _ = seq.attend(q, 0.01, 0.7)
+    assert not sel.any()
+    if kind == "q2":
+        ref = _sdpa(q, seq.qk.dequant(), seq.qv.dequant_full(), 0.7)
+    else:
+        ref = _sdpa(q, k, v, 0.7)
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("tau", [1e-3, 1e-2, 5e-2])
+def test_general_tau_decomposition(tau):
+    q, k, v, seq = _case(4, n=517, q_scale=3.0)
+    o, sel, p = seq.attend(q, tau, 1.0)
+    kh, vf, vh = seq.qk.dequant(), seq.qv.dequant_full(), seq.qv.dequant_high()
+    pt = _torch_p(q, kh, 1.0)
+    np.testing.assert_allclose(p, pt, rtol=1e-12, atol=1e-15)
+    want_sel = pt.astype(np.float32) >= np.float32(tau)
+    np.testing.assert_array_equal(sel, want_sel)
+    ref = _sdpa(q, kh, vh, 1.0) + (pt[want_sel, None] * (vf - vh)[want_sel]).sum(axis=0)
+    np.testing.assert_allclose(o, ref, rtol=1e-10, atol=1e-12)
+    assert 0 < sel.sum() < sel.size
+
+
+def test_selection_invariants():
+    q, k, v, seq = _case(5, n=1000, q_scale=4.0)
+    prev = None
+    for tau in [0.0, 1e-4, 1e-3, 3e-3, 1e-2, 5e-2, 0.2, 1.0, math.inf]:
+        _, sel, _ = seq.attend(q, tau, 1.0)
+        if 0 < tau < math.inf:
+            assert sel.sum() <= math.floor(1 / tau)
+        if prev is not None:
+            assert np.all(sel <= prev)          # larger tau selects a subset
+        prev = sel
+
+
+def test_output_inside_value_hull():
+    q, k, v, seq = _case(6, n=200, q_scale=2.0)
+    o, sel, _ = seq.attend(q, 0.01, 1.0)
+    vhat = np.where(sel[:, None], seq.qv.dequant_full(), seq.qv.dequant_high())
+    assert np.all(o >= vhat.min(axis=0) - 1e-12) and np.all(o <= vhat.max(axis=0) + 1e-12)
+
+
+def test_single_token_returns_its_full_value():
+    q, k, v, seq = _case(7, n=1)
+    o, sel, p = seq.attend(q, 0.5, 1.0)
+    assert sel.tolist() == [True] and p.tolist() == [1.0]
+    np.testing.assert_allclose(o, seq.qv.dequant_full()[0], rtol=0, atol=0)
+
+
+def test_zero_query_is_uniform_average():
+    q, k, v, seq = _case(8, n=64)
+    q = np.zeros_like(q)
+    o, sel, p = seq.attend(q, 1 / 64, 1.0)       # p = 1/64 >= tau: all selected
+    assert sel.all()
+    np.testing.assert_allclose(o, seq.qv.dequant_full().mean(axis=0), rtol=1e-12)
+    o2, sel2, _ = seq.attend(q, 1 / 63, 1.0)     # p < tau: none selected
+    assert not sel2.any()
+    np.testing.assert_allclose(o2, seq.qv.dequant_high().mean(axis=0), rtol=1e-12)
+
+
+def test_sm_scale_equals_scaled_query():
+    q, k, v, seq = _case(9, n=100, kind="q2")
+    o1, _, _ = seq.attend(q, 0.0, 0.25)
+    o2, _, _ = seq.attend(q * np.float32(0.25), 0.0, 1.0)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12)
+
+
+def test_empty_sequence_gives_zeros():
+    o, sel, p = O.attend(np.ones(64), np.zeros((0, 64)), np.zeros((0, 64)), None, 0.1, 1.0)
+    assert o.shape == (64,) and not o.any() and sel.size == 0
+
+
+def test_reuse_reads_final_loop_with_own_query():
+    rng = np.random.default_rng(10)
+    L, N, H, B, n, d = 2, 2, 1, 1, 70, 64
+    plan = ["reuse", "q2", "q4", "q4"]
+    stored = {}
+    for cell in (1, 2, 3):
+        k, v = _bf16(rng, (n, d)), _bf16(rng, (n, d))
+        stored[(cell, 0, 0)] = O.StoredSequence(plan[cell], k, v)
+    q = _bf16(rng, (B, H, d), 2.0)
+    got = O.decode_cell(plan, N, 0, stored, q, [n], 0.02, 1.0, pairs=[(0, 0)])[(0, 0)]
+    want = stored[(2, 0, 0)].attend(q[0, 0], 0.02, 1.0)
+    np.testing.assert_array_equal(got[0], want[0])
+    np.testing.assert_array_equal(got[1], want[1])
+    assert O.resolve_source(plan, 1, N) == 1
+    with pytest.raises(ValueError):
+        O.resolve_source(["q4", "reuse"], 1, 1)
+
+
+def test_brute_force_tiny_loops():
+    """Explicit scalar loops over tokens and channels (math.exp, Python
+    floats) against the vectorised oracle on a tiny 4-bit case."""
+    rng = np.random.default_rng(11)
+    n, d, tau = 40, 32, 0.03
+    k, v = _bf16(rng, (n, d)), _bf16(rng, (n, d))
+    q = _bf16(rng, (d,), 2.0)
+    seq = O.StoredSequence("q4", k, v)
+    o, sel, _ = seq.attend(q, tau, 1.0)
+    qk, qv = seq.qk, seq.qv
+    logits = []
+    for t in range(n):
+        acc = 0.0
+        for c in range(d):
+            if t < 32:
+                kv = float(qk.minv[0, c]) + float(qk.scale[0, c]) * int(qk.codes[t, c])
+            else:
+                kv = float(k[t, c])
+            acc += float(q[c]) * kv
+        logits.append(acc)
+    m = max(logits)
+    e = [math.exp(s - m) for s in logits]
+    z = sum(e)
+    out = [0.0] * d
+    for t in range(n):
+        p = e[t] / z
+        take_low = np.float32(p) >= np.float32(tau)
+        assert take_low == sel[t]
+        for c in range(d):
+            code = int(qv.codes[t, c])
+            s, mn = float(qv.scale[t, 0]), float(qv.minv[t, 0])
+            val = mn + s * (code if take_low else 4 * (code >> 2) + 1.5)
+            out[c] += p * val
+    np.testing.assert_allclose(o, out, rtol=1e-11, atol=1e-13)
+
+
+def test_dequantised_cache_within_round_trip_bound():
+    """Dequantised keys and values stay within the quantiser's closed-form
+    error bound of the bf16 inputs (half a step, or the top overshoot)."""
+    q, k, v, seq = _case(12, n=333, d=64)
+    kh, vf = seq.qk.dequant(), seq.qv.dequant_full()
+    ks = np.repeat(seq.qk.scale.astype(np.float64), 32, axis=0)      # [320, d]
+    k_top = np.repeat((k[:320].reshape(10, 32, 64).max(axis=1)
+                       - (seq.qk.minv + 15.0 * seq.qk.scale.astype(np.float64))), 32, axis=0)
+    kb = np.maximum(ks / 2, k_top) * (1 + 1e-6) + 1e-6
+    assert np.all(np.abs(kh[:320] - k[:320]) <= kb)
+    np.testing.assert_array_equal(kh[320:], k[320:])
+    vs = np.repeat(seq.qv.scale.astype(np.float64), 32, axis=1)
+    v_top = np.repeat(v.reshape(333, 2, 32).max(axis=2)
+                      - (seq.qv.minv + 15.0 * seq.qv.scale.astype(np.float64)), 32, axis=1)
+    vb = np.maximum(vs / 2, v_top) * (1 + 1e-6) + 1e-6
+    assert np.all(np.abs(vf - v) <= vb)
+
+
+def test_high_plane_value_is_bucket_midpoint():
+    """The high-plane-only value is the mean of the four full-precision
+    values that share its high bits (unbiased for uniform low bits)."""
+    q, k, v, seq = _case(13, n=50)
+    qv = seq.qv
+    s = np.repeat(qv.scale.astype(np.float64), 32, axis=1)
+    m = np.repeat(qv.minv.astype(np.float64), 32, axis=1)
+    hi = (qv.codes >> 2).astype(np.float64)
+    bucket = np.mean([m + s * (4 * hi + lo) for lo in range(4)], axis=0)
+    np.testing.assert_allclose(qv.dequant_high(), bucket, rtol=1e-15, atol=1e-15)
+    assert np.all(np.abs(qv.dequant_full() - qv.dequant_high()) <= 1.5 * s + 1e-12)
