@@ -1,0 +1,473 @@
+#!/usr/bin/env python3
+"""Benchmark of the LoopKV decode path on B200.
+
+Metric: decode-attention KV GB/s (algorithmic bytes the decode kernels must
+move, over device time) and microseconds per looped decode step.
+
+One step = every (loop, layer) cell of the Ouro-1.4B-like workload in order:
+stored cells append the current token (quantise-append kernel) and attend
+over n + 1 tokens, reuse cells attend over the final loop's n tokens (fused
+decode-attention kernel).  The step is captured once in a CUDA graph (kernels
+launched with programmatic dependent launch) and replayed.  Every step
+decodes at the same position (the append rewrites the same token), so the
+context stays at the workload's length however many steps are timed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank holds its own batch
+(sequence data parallelism, no collective on the data path); the timed
+region is bracketed by barriers and the slowest rank's time is used.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention KV GB/s (% of B200 HBM peak) and µs per looped decode step"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    ap.add_argument("--workload", default="ouro_step")
+    ap.add_argument("--splits", type=int, default=0, help="decode splits override (0 = automatic)")
+    ap.add_argument("--no-pdl", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------- ranks
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, local, backend="nccl"):
+    if world <= 1:
+        return
+    import torch.distributed as dist
+    kw = dict(backend=backend, timeout=datetime.timedelta(seconds=120))
+    if backend == "nccl":
+        kw["device_id"] = torch.device(f"cuda:{local}")
+    dist.init_process_group(**kw)
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of x over all ranks (the slowest rank's time)."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(bytes_per_rank: float, world: int, seconds_max: float) -> float:
+    """Whole-job GB/s: bytes all ranks moved over the slowest rank's time."""
+    return bytes_per_rank * world / seconds_max / 1e9
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons of one GPU (NVML) while the
+    timed region runs.  Reads only; changes no GPU setting."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(f"GPU-{props.uuid}")
+            except Exception:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report no clocks
+            self._nv, self.error = None, str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for mask, name in self.REASONS.items():
+                    if bits & mask:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if self._nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- peaks, profile
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("decode.cu", "device_common.cuh"):
+        with open(os.path.join(ROOT, "mixed_precision_kv_loopkv_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"decode_attention_{workload}.md")
+    try:
+        fields = {}
+        for line in open(path):
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+        if fields.get("source_sha256") != decode_source_hash():
+            return None
+        return float(fields["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- workload setup
+
+def setup(w, pdl: bool, splits: int, extra: int = 64):
+    from mixed_precision_kv_loopkv_b200 import (LOOPKV_FLAG_PDL, KVCells, LoopedDecodeStep,
+                                                loopkv_quantize_append)
+    from workload import block_table_for, cell_kv, cell_new_token, cell_query, make_plan, seq_lens_for
+
+    plan = make_plan(w)
+    lens = seq_lens_for(w)
+    table_np, num_blocks = block_table_for(w, lens + extra)
+    kv = KVCells(plan, w.num_loops, w.num_layers, w.num_heads, w.head_dim, num_blocks, w.batch,
+                 table_np.shape[1], flags=LOOPKV_FLAG_PDL if pdl else 0, decode_splits=splits)
+    table = torch.from_numpy(table_np).cuda()
+    zero = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
+    stored = [c for c, k in enumerate(plan) if k != "reuse"]
+    for c in stored:
+        loop, layer = divmod(c, w.num_layers)
+        k, v = cell_kv(w, loop, layer, device="cuda")
+        loopkv_quantize_append(kv, loop, layer, k, v, table, zero)
+        del k, v
+    C = len(plan)
+    q_all = torch.stack([cell_query(w, *divmod(c, w.num_layers), device="cuda") for c in range(C)])
+    kn_all = torch.empty((len(stored), w.batch, 1, w.num_heads, w.head_dim), dtype=torch.bfloat16,
+                         device="cuda")
+    vn_all = torch.empty_like(kn_all)
+    for i, c in enumerate(stored):
+        kn_all[i], vn_all[i] = cell_new_token(w, *divmod(c, w.num_layers), device="cuda")
+    out_all = torch.zeros_like(q_all)
+    sel_all = torch.zeros((C, w.batch, w.num_heads), dtype=torch.int32, device="cuda")
+    slot = {c: i for i, c in enumerate(stored)}
+    pos = torch.from_numpy(lens).cuda()
+    step = LoopedDecodeStep(
+        kv, table, pos, [q_all[c] for c in range(C)],
+        {c: kn_all[slot[c]] for c in stored}, {c: vn_all[slot[c]] for c in stored},
+        [out_all[c] for c in range(C)], w.tau, w.sm_scale, int(lens.max()) + 1,
+        sel_count=[sel_all[c] for c in range(C)])
+    torch.cuda.synchronize()
+    return dict(plan=plan, lens=lens, kv=kv, step=step, q_all=q_all, kn_all=kn_all, vn_all=vn_all,
+                out_all=out_all, sel_all=sel_all)
+
+
+class DecodeOnly:
+    """The decode launches of a step without the appends (roofline timing)."""
+
+    def __init__(self, step):
+        self.s = step
+
+    def run(self):
+        from mixed_precision_kv_loopkv_b200 import LOOPKV_CELL_REUSE, loopkv_decode_attention
+        s, kv = self.s, self.s.kv
+        for cell in s.cells:
+            loop, layer = divmod(cell, kv.num_layers)
+            lens = s.pos if kv.plan_codes[cell] == LOOPKV_CELL_REUSE else s.pos_next
+            loopkv_decode_attention(kv, loop, layer, s.q[cell], s.block_table, lens, s.tau, s.sm_scale,
+                                    out=s.out[cell], max_seq_len=s.max_seq_len,
+                                    sel_count=s.sel_count[cell])
+
+
+def capture(fn):
+    fn()                     # eager warm-up (idempotent at a fixed position)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def time_replays(g, n: int) -> float:
+    """Device milliseconds of n back-to-back replays (events on this stream)."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n):
+        g.replay()
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b)
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, plan, lens, n_pairs: int, seed: int = 0):
+    """A seeded sample of (cell, sequence, head) decodes for the CPU oracle:
+    the same inputs as the GPU run, built into the oracle's own stored form."""
+    import oracle as O
+    from workload import cell_kv, cell_query
+    rng = np.random.default_rng(seed)
+    C = len(plan)
+    cells = rng.choice(C, size=min(n_pairs, C), replace=False)
+    items = []
+    for cell in cells:
+        cell = int(cell)
+        src = cell if plan[cell] != "reuse" else (w.num_loops - 1) * w.num_layers + cell % w.num_layers
+        b, h = int(rng.integers(w.batch)), int(rng.integers(w.num_heads))
+        n = int(lens[b])
+        k, v = cell_kv(w, *divmod(src, w.num_layers), device="cuda")
+        kk = k[b, :n, h].float().cpu().numpy()
+        vv = v[b, :n, h].float().cpu().numpy()
+        del k, v
+        q = cell_query(w, *divmod(cell, w.num_layers), device="cuda")[b, h].float().cpu().numpy()
+        items.append((plan[src], O.StoredSequence(plan[src], kk, vv), q, n))
+    torch.cuda.empty_cache()
+    return items
+
+
+def run_oracle(items, w, budget_s: float = None, steps: int = None, warmup: int = 0):
+    """Time the oracle's decode over the sample (one item per step, round
+    robin); returns (GB/s, seconds, items run, threads)."""
+    from threadpoolctl import threadpool_limits
+    from mixed_precision_kv_loopkv_b200.accounting import decode_bytes
+    total_bytes, n_run = 0, 0
+    with threadpool_limits(limits=1):
+        torch_threads = torch.get_num_threads()
+        torch.set_num_threads(1)
+        try:
+            for i in range(warmup):
+                kind, seq, q, n = items[i % len(items)]
+                seq.attend(q, w.tau, w.sm_scale)
+            t0 = time.perf_counter()
+            i = 0
+            while True:
+                kind, seq, q, n = items[i % len(items)]
+                o, sel, _ = seq.attend(q, w.tau, w.sm_scale)
+                total_bytes += decode_bytes(kind, w.head_dim, n, int(sel.sum()))
+                i += 1
+                el = time.perf_counter() - t0
+                if steps is not None and i >= steps:
+                    break
+                if budget_s is not None and el >= budget_s:
+                    break
+            n_run = i
+        finally:
+            torch.set_num_threads(torch_threads)
+    return total_bytes / el / 1e9, el, n_run, 1
+
+
+# ----------------------------------------------------------------- arms
+
+def workload_config(w, world):
+    frac = f"{round(w.frac_q4 * 100)}/{round((1 - w.frac_q4 - w.frac_reuse) * 100)}/{round(w.frac_reuse * 100)}"
+    ctx = f"{w.ctx_range[0]}..{w.ctx_range[1]}" if w.ctx_range else str(w.context)
+    return {
+        "workload": (f"{w.name}: batch {w.batch}, {w.num_loops} loops x {w.num_layers} layers, "
+                     f"{w.num_heads} MHA heads x {w.head_dim}, context {ctx}, plan {frac} "
+                     f"4b/2b/reuse, tau {w.tau}, paged 16-token blocks ({w.paging})"),
+        "batch_per_gpu": w.batch, "context": ctx, "cells": w.num_cells, "tau": w.tau,
+        "l2": "inputs larger than L2 (whole step streams the cache once)",
+        "parallelism": f"dp{world} (sequences)",
+    }
+
+
+def reference_arm(args, world, rank):
+    """The oracle as it stands on the host cores, one sampled (cell,
+    sequence, head) decode per step."""
+    from workload import get_workload, make_plan, seq_lens_for
+    if rank != 0:
+        return
+    w = get_workload(args.workload)
+    plan, lens = make_plan(w), seq_lens_for(w)
+    items = oracle_sample(w, plan, lens, n_pairs=16)
+    gbs, secs, n_run, cores = run_oracle(items, w, steps=args.steps, warmup=args.warmup)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(n_run, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, 1),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"one (cell, sequence, head) decode per step, round robin over 16 "
+                                   f"seeded pairs of the {w.name} workload"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main_arm(args, world, rank, local):
+    from mixed_precision_kv_loopkv_b200.accounting import step_bytes
+    from workload import get_workload
+
+    torch.cuda.set_device(local)
+    init_dist(world, local)
+    w = get_workload(args.workload)
+    S = setup(w, pdl=not args.no_pdl, splits=args.splits)
+    step, plan, lens = S["step"], S["plan"], S["lens"]
+    dev = torch.device(f"cuda:{local}")
+
+    g = capture(step.run)
+    for _ in range(max(args.warmup, 3)):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        ms = time_replays(g, args.steps)
+    barrier(world)
+    ms_max = max_over_ranks(ms, world, dev)
+
+    sel = S["sel_all"].cpu().numpy()
+    bytes_step = step_bytes(plan, w.num_layers, w.num_loops, w.head_dim, w.num_heads, lens + 1, lens, sel)
+    value = aggregate_value(bytes_step * args.steps, world, ms_max / 1e3)
+    us_step = ms_max / args.steps * 1e3
+
+    # dominant kernel: the decode launches alone, same state
+    gd = capture(DecodeOnly(step).run)
+    reps = max(20, args.steps // 4)
+    ms_dec = time_replays(gd, reps)
+    launches = len(step.cells)
+    per_launch_s = ms_dec / 1e3 / (reps * launches)
+    achieved = bytes_step / launches / per_launch_s / 1e9
+    peak, peak_kind = hbm_peak()
+    traffic = profiled_traffic(w.name)
+
+    # end to end: inputs of every step copied in from pinned host memory,
+    # outputs copied back, inside the timed region
+    q_h = S["q_all"].cpu().pin_memory()
+    kn_h = S["kn_all"].cpu().pin_memory()
+    vn_h = S["vn_all"].cpu().pin_memory()
+    out_h = torch.empty(S["out_all"].shape, dtype=S["out_all"].dtype).pin_memory()
+    e2e_steps = max(3, args.steps // 4)
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(e2e_steps):
+        S["q_all"].copy_(q_h, non_blocking=True)
+        S["kn_all"].copy_(kn_h, non_blocking=True)
+        S["vn_all"].copy_(vn_h, non_blocking=True)
+        g.replay()
+        out_h.copy_(S["out_all"], non_blocking=True)
+    b.record()
+    b.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    h2d = q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2
+    d2h = out_h.numel() * 2
+    e2e_value = aggregate_value(bytes_step * e2e_steps, world, e2e_ms / 1e3)
+
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        items = oracle_sample(w, plan, lens, n_pairs=12)
+        gbs, secs, n_run, cores = run_oracle(items, w, budget_s=args.cpu_seconds, warmup=2)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"{n_run} (cell, sequence, head) decodes over {secs:.1f} s, round robin over "
+                         f"12 seeded pairs of the {w.name} workload (numpy fp64, one BLAS thread)"}
+
+    if rank == 0:
+        cfg = workload_config(w, world)
+        cfg.update({"pdl": not args.no_pdl, "splits": args.splits or "auto", "cuda_graph": True,
+                    "algorithmic_bytes_per_step": bytes_step,
+                    "selected_low_plane_rows_per_step": int(sel.sum())})
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": us_step / 1e3, "us_per_step": us_step,
+            "pct_of_hbm_peak": value / world / peak * 100, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "decode_kernel (all decode launches of one step, timed alone)",
+                         "per_launch_us": per_launch_s * 1e6,
+                         "bytes_per_launch": bytes_step / launches,
+                         "peak_source": f"{peak_kind} hbm_gbs"},
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "us_per_step": e2e_ms / e2e_steps * 1e3},
+            "gpu_launches": args.steps * step.launches_per_step(),
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del g, gd
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        return
+    main_arm(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

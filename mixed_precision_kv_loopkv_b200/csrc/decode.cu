@@ -1,0 +1,701 @@
+// Fused LoopKV decode attention (sm_100a).
+//
+// LoopKV: Loop-Aware KV Cache Compression for Serving Looped Transformers,
+// Abstract: each (loop, layer) cell is read at its planned precision (4-bit,
+// 2-bit, or the final loop's cell reused); every token's high 2-bit value
+// plane is read, and the low plane only where the cell's own attention
+// weights need 4-bit precision; one fused kernel executes the plan.  The
+// threshold reading used here: token t takes its low plane when its fp32
+// softmax weight p_t >= tau.  Split-K over the context follows the
+// streaming-softmax idea (O(1)-memory attention in the same pages' listing).
+//
+// Grid (splits, heads, batch); the splits of one (sequence, head) form one
+// thread-block cluster.  Each CTA:
+//   - a producer lane streams the pass-1 prefix of every block record of its
+//     context chunk (keys, key meta, value high plane, value meta: 2048 B of
+//     the 2560-B 4-bit record at D = 128) with 1-D bulk copies (TMA, no
+//     multicast) into an NS-stage shared-memory ring;
+//   - NW consumer warps each take whole 32-token groups: dequantise the keys
+//     at the cell's precision, form the logits, keep an online softmax and
+//     accumulate the high-plane values;
+//   - the splits exchange (max, sum) through distributed shared memory, so
+//     every CTA knows the exact normaliser Z before any low-plane read;
+//   - pass 2 re-reads the CTA's logits from shared memory, ballots the tokens
+//     with p >= tau and gathers only their 32-byte low-plane rows, adding
+//     p * scale * (lo - 1.5) per channel (turning the bucket midpoint into
+//     the full 4-bit value);
+//   - a cluster-wide reduction over distributed shared memory writes bf16 out.
+//
+// Arithmetic for the HBM-bound inner loop (one FP32x2 FMA per two elements):
+// a code's bits are isolated in place with one AND and read as an fp32
+// subnormal, code * 2^pos * 2^-149; the per-channel factor 2^(149 - pos - E)
+// is folded into the query (keys) or undone once per channel at the end
+// (values).  Subnormal FMA inputs are exact on this hardware (no FTZ), so
+// every product equals q * scale * code up to the global power of two 2^-E.
+#include <float.h>
+
+#include <algorithm>
+
+#include "device_common.cuh"
+#include "kernels.h"
+
+namespace loopkv {
+namespace {
+
+constexpr int kNW = 4;        // consumer warps per CTA
+constexpr int kThreads = 32 * (kNW + 1);
+constexpr int kExpOff = 64;   // E: products live at 2^-64 of their true size
+
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// Field position (bits) of channel i of a 16-channel chunk.
+// 2-bit plane word: channel i at bits 2i; i >= 11 is read from (w >> 22).
+__device__ __forceinline__ constexpr int pos2(int i) { return 2 * (i < 11 ? i : i - 11); }
+// 4-bit nibble words (even/odd channels): channel i in nibble i/2;
+// nibbles >= 5 are read from (w >> 20).
+__device__ __forceinline__ constexpr int pos4(int i) { return 4 * ((i >> 1) < 5 ? (i >> 1) : (i >> 1) - 5); }
+
+// Subnormal view of field i of a 2-bit plane word.
+__device__ __forceinline__ float fld2(uint32_t w, uint32_t w22, int i) {
+  return i < 11 ? __uint_as_float(w & (3u << (2 * i))) : __uint_as_float(w22 & (3u << (2 * (i - 11))));
+}
+// Subnormal view of nibble m of a nibble word.
+__device__ __forceinline__ float nib(uint32_t w, uint32_t w20, int m) {
+  return m < 5 ? __uint_as_float(w & (15u << (4 * m))) : __uint_as_float(w20 & (15u << (4 * (m - 5))));
+}
+// Full 4-bit codes of 16 channels from their high and low plane words:
+// even = channels 0,2,..,14 in nibbles 0..7; odd = channels 1,3,..,15.
+__device__ __forceinline__ void combine_planes(uint32_t hi, uint32_t lo, uint32_t& even, uint32_t& odd) {
+  even = ((hi << 2) & 0xCCCCCCCCu) | (lo & 0x33333333u);
+  odd = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
+}
+
+// Dot product of 16 subnormal code views with 16 pre-scaled coefficients.
+template <bool FOUR>
+__device__ __forceinline__ float dot16(const float* c, uint32_t a, uint32_t b, float init) {
+  float2 acc = make_float2(init, 0.f);
+  if constexpr (FOUR) {  // a, b = even/odd nibble words
+    uint32_t e, o;
+    combine_planes(a, b, e, o);
+    const uint32_t e20 = e >> 20, o20 = o >> 20;
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      acc = __ffma2_rn(make_float2(c[2 * m], c[2 * m + 1]), make_float2(nib(e, e20, m), nib(o, o20, m)), acc);
+  } else {  // a = 2-bit plane word
+    const uint32_t a22 = a >> 22;
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+      acc = __ffma2_rn(make_float2(c[2 * p], c[2 * p + 1]),
+                       make_float2(fld2(a, a22, 2 * p), fld2(a, a22, 2 * p + 1)), acc);
+  }
+  return acc.x + acc.y;
+}
+
+// acc[p] += w * (codes 2p, 2p+1)
+template <bool FOUR>
+__device__ __forceinline__ void axpy16(float2* acc, float w, uint32_t a, uint32_t b) {
+  const float2 ww = make_float2(w, w);
+  if constexpr (FOUR) {
+    uint32_t e, o;
+    combine_planes(a, b, e, o);
+    const uint32_t e20 = e >> 20, o20 = o >> 20;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) acc[m] = __ffma2_rn(ww, make_float2(nib(e, e20, m), nib(o, o20, m)), acc[m]);
+  } else {
+    const uint32_t a22 = a >> 22;
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+      acc[p] = __ffma2_rn(ww, make_float2(fld2(a, a22, 2 * p), fld2(a, a22, 2 * p + 1)), acc[p]);
+  }
+}
+
+template <int KIND, int D, bool FULLV>
+struct Cfg {
+  using R = Rec<KIND, D>;
+  static constexpr bool kQuant = KIND != LOOPKV_CELL_BF16;
+  static constexpr bool kQ4 = KIND == LOOPKV_CELL_Q4;
+  // bytes of one block record streamed in pass 1
+  static constexpr int kLoad = kQ4 ? (FULLV ? R::kBytes : R::kQ4VLo) : R::kBytes;
+  static constexpr int kStage = 2 * kLoad;                 // one 32-token group
+  static constexpr int kNS = kQuant ? 8 : 4;               // ring stages
+  static constexpr int kCH = D / 16;                       // lanes per token
+  static constexpr int kTS = 32 / kCH;                     // token sub-groups per warp
+  static constexpr int kTPL = kCH;                         // tokens per lane per group
+  static constexpr int kE = kQuant ? kExpOff : 0;
+  static constexpr bool kLogits = kQ4 && !FULLV;           // pass 2 needs the logits
+};
+
+// Shared-memory carve-up (bytes), identical on host and device.
+struct Smem {
+  size_t stages, bars, ids, logits, wscr, cta, total;
+};
+__host__ __device__ inline Smem smem_plan(int stage_bytes, int ns, int cg, int d, bool logits) {
+  Smem s;
+  s.stages = 0;
+  s.bars = s.stages + static_cast<size_t>(stage_bytes) * ns;
+  s.ids = s.bars + 16 * ns;
+  s.logits = s.ids + ((8 * cg + 15) / 16) * 16;
+  s.wscr = s.logits + (logits ? 128 * static_cast<size_t>(cg) : 0);
+  s.cta = s.wscr + static_cast<size_t>(kNW) * (d + 4) * 4;
+  s.total = s.cta + static_cast<size_t>(d + 4) * 4;
+  return s;
+}
+
+// Per-CTA scalar slots in the cta segment after the D accumulators.
+enum { kSlotM = 0, kSlotL = 1, kSlotCount = 2, kSlotBad = 3 };
+
+template <int KIND, int D, bool FULLV, bool CLUSTER>
+__global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
+  using C = Cfg<KIND, D, FULLV>;
+  using R = typename C::R;
+  constexpr int CH = C::kCH, TS = C::kTS, TPL = C::kTPL, NS = C::kNS;
+  constexpr int LOAD = C::kLoad, STAGE = C::kStage;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const Smem sp = smem_plan(STAGE, NS, p.chunk_groups, D, C::kLogits);
+  uint8_t* stages = smem + sp.stages;
+  const uint32_t full_bar = smem_addr(smem + sp.bars);
+  const uint32_t empty_bar = full_bar + 8 * NS;
+  int32_t* ids = reinterpret_cast<int32_t*>(smem + sp.ids);
+  float* logits = reinterpret_cast<float*>(smem + sp.logits);
+  float* wscr = reinterpret_cast<float*>(smem + sp.wscr);
+  float* cta_acc = reinterpret_cast<float*>(smem + sp.cta);
+  float* cta_f = cta_acc + D;
+  int* cta_i = reinterpret_cast<int*>(cta_f);
+
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int S = gridDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_allow_dependents();
+
+  // ---- this split's chunk of 32-token groups
+  const int n = p.seq_lens[b];
+  int bad = 0;
+  if (n < 0 || n > p.max_seq_len || n > p.max_blocks * kBlock) bad = LOOPKV_DEVERR_SEQ_LEN;
+  const int nn = bad ? 0 : n;
+  const int ng = (nn + kGroup - 1) / kGroup;
+  const int per = (ng + S - 1) / S;
+  const int g0 = min(split * per, ng);
+  const int cg = min(per, ng - g0);
+  if (cg > p.chunk_groups) bad = LOOPKV_DEVERR_SEQ_LEN;
+  const int n_blocks = (nn + kBlock - 1) / kBlock;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(full_bar + 8 * i, 1);
+      mbar_init(empty_bar + 8 * i, 1);
+    }
+    cta_f[kSlotM] = -INFINITY;
+    cta_f[kSlotL] = 0.f;
+    cta_i[kSlotCount] = 0;
+    cta_i[kSlotBad] = bad;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == kNW && !bad) {
+    for (int i = lane; i < 2 * cg; i += 32) {
+      const int lb = 2 * g0 + i;
+      int id = -1;
+      if (lb < n_blocks) {
+        id = p.block_table[static_cast<size_t>(b) * p.max_blocks + lb];
+        if (id < 0 || id >= p.num_blocks) atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_BLOCK_ID);
+      }
+      ids[i] = id;
+    }
+  }
+  __syncthreads();
+  bad = cta_i[kSlotBad];
+
+  // ---- pass 1
+  const int k = lane % CH, r = lane / CH;
+  float m_w = -INFINITY, l_w = 0.f, beta = 0.f;
+  float2 acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = make_float2(0.f, 0.f);
+
+  if (!bad && cg > 0) {
+    if (warp == kNW) {
+      if (lane == 0) {
+        // producer: blocks of groups before the one holding the newest token
+        // cannot be written by the previous kernel, so they stream at once.
+        const uint64_t pol = l2_evict_first_policy();
+        const int g_unsafe = (nn - 1) / kGroup;
+        bool waited = false;
+        for (int gi = 0; gi < cg; ++gi) {
+          const int stage = gi % NS;
+          if (gi >= NS && !mbar_wait(empty_bar + 8 * stage, ((gi / NS) - 1) & 1)) {
+            atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_TIMEOUT);
+            break;
+          }
+          const int G = g0 + gi;
+          if (!waited && G >= g_unsafe) {
+            pdl_wait_prior_grid();
+            waited = true;
+          }
+          const int nb = min(2, n_blocks - 2 * G);
+          mbar_arrive_expect_tx(full_bar + 8 * stage, nb * LOAD);
+          for (int blk = 0; blk < nb; ++blk)
+            bulk_load(smem_addr(stages + stage * STAGE + blk * LOAD),
+                      p.arena + (static_cast<size_t>(ids[2 * gi + blk]) * p.H + h) * R::kBytes,
+                      LOAD, full_bar + 8 * stage, pol);
+        }
+      }
+    } else {
+      pdl_wait_prior_grid();  // q and the key residual may come from the previous kernel
+      // this lane's 16 query channels, in log2 units
+      float qf[16], qs[16];
+      {
+        const uint4* qp = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.H + h) * D + 16 * k);
+        const uint4 a = qp[0], c = qp[1];
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          qf[2 * i] = bf16_lo(w[i]) * p.sm_scale_log2;
+          qf[2 * i + 1] = bf16_hi(w[i]) * p.sm_scale_log2;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          qs[i] = qf[i] * pow2i(149 - (C::kQ4 ? pos4(i) : pos2(i)) - C::kE);
+      }
+      const float esc = pow2i(C::kE), inv_esc = pow2i(-C::kE);
+
+      for (int gi = warp; gi < cg; gi += kNW) {
+        const int stage = gi % NS;
+        if (!mbar_wait(full_bar + 8 * stage, (gi / NS) & 1)) {
+          atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_TIMEOUT);
+          break;
+        }
+        const uint8_t* st = stages + stage * STAGE;
+        const int tok0 = (g0 + gi) * kGroup;
+        const bool tail = tok0 + kGroup > nn;
+
+        // ---- keys -> logits (scaled by 2^-E)
+        float part[TPL];
+        if constexpr (C::kQuant) {
+          if (!tail) {
+            const uint8_t* km = st + ((16 * k < D / 2) ? 0 : LOAD) + R::kKMetaOff + ((16 * k) % (D / 2)) * 4;
+            float q2[16];
+            float alpha = 0.f;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint4 mw = reinterpret_cast<const uint4*>(km)[v];
+              const uint32_t ws[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int i = 4 * v + u;
+                q2[i] = qs[i] * bf16_lo(ws[u]);
+                alpha = fmaf(qf[i], bf16_hi(ws[u]), alpha);
+              }
+            }
+            alpha *= inv_esc;
+#pragma unroll
+            for (int j = 0; j < TPL; ++j) {
+              const int t = r + TS * j;
+              const uint8_t* row = st + (t >> 4) * LOAD + (t & 15) * R::kRow + 4 * k;
+              const uint32_t w0 = *reinterpret_cast<const uint32_t*>(row + R::kKHi);
+              if constexpr (C::kQ4) {
+                const uint32_t w1 = *reinterpret_cast<const uint32_t*>(row + R::kQ4KLo);
+                part[j] = dot16<true>(q2, w0, w1, alpha);
+              } else {
+                part[j] = dot16<false>(q2, w0, 0u, alpha);
+              }
+            }
+          } else {
+            // unfinished key group: exact bf16 keys from the residual
+            const __nv_bfloat16* res = p.residual + (static_cast<size_t>(b) * p.H + h) * kGroup * D + 16 * k;
+#pragma unroll
+            for (int j = 0; j < TPL; ++j) {
+              const int t = r + TS * j;
+              float d = 0.f;
+              if (tok0 + t < nn) {
+                const uint4* kp = reinterpret_cast<const uint4*>(res + t * D);
+                const uint4 a = kp[0], c = kp[1];
+                const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+                float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  s2 = __ffma2_rn(make_float2(qf[2 * i], qf[2 * i + 1]), make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
+                d = (s2.x + s2.y) * inv_esc;
+              }
+              part[j] = d;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < TPL; ++j) {
+            const int t = r + TS * j;
+            const uint4* kp = reinterpret_cast<const uint4*>(st + (t >> 4) * LOAD + R::kBfK + (t & 15) * D * 2 + 32 * k);
+            const uint4 a = kp[0], c = kp[1];
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+            float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              s2 = __ffma2_rn(make_float2(qf[2 * i], qf[2 * i + 1]), make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
+            part[j] = s2.x + s2.y;
+          }
+        }
+        // all-reduce each token's logit over its CH lanes
+#pragma unroll
+        for (int j = 0; j < TPL; ++j)
+#pragma unroll
+          for (int o = 1; o < CH; o <<= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+
+        // ---- online softmax over the group (log2 units)
+        float gm = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < TPL; ++j)
+          if (tok0 + r + TS * j < nn) gm = fmaxf(gm, part[j]);
+#pragma unroll
+        for (int o = CH; o < 32; o <<= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+        gm *= esc;
+        if (gm > m_w) {
+          const float c = fast_exp2(m_w - gm);
+          l_w *= c;
+          beta *= c;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = make_float2(acc[i].x * c, acc[i].y * c);
+          m_w = gm;
+        }
+        float wgt[TPL];
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) {
+          wgt[j] = (tok0 + r + TS * j < nn) ? fast_exp2(fmaf(part[j], esc, -m_w)) : 0.f;
+          l_w += wgt[j];
+        }
+        if constexpr (C::kLogits) {
+          float mine = part[0];
+#pragma unroll
+          for (int j = 1; j < TPL; ++j) mine = (j == k) ? part[j] : mine;
+          logits[gi * kGroup + r + TS * k] = mine * esc;
+        }
+
+        // ---- values
+#pragma unroll
+        for (int j = 0; j < TPL; ++j) {
+          const int t = r + TS * j;
+          if constexpr (C::kQuant) {
+            const uint8_t* blk = st + (t >> 4) * LOAD;
+            const uint32_t mv = *reinterpret_cast<const uint32_t*>(blk + R::kVMetaOff + ((t & 15) * (D / kGroup) + (k >> 1)) * 4);
+            const bool ok = !tail || (tok0 + t < nn);
+            const float s = ok ? bf16_lo(mv) : 0.f;
+            const float mn = ok ? bf16_hi(mv) : 0.f;
+            const uint8_t* row = blk + (t & 15) * R::kRow + 4 * k;
+            const uint32_t vh = *reinterpret_cast<const uint32_t*>(row + R::kVHi);
+            if constexpr (C::kQ4 && FULLV) {
+              const uint32_t vl = *reinterpret_cast<const uint32_t*>(row + R::kQ4VLo);
+              beta = fmaf(wgt[j], mn, beta);
+              axpy16<true>(acc, wgt[j] * s * pow2i(85), vh, vl);
+            } else if constexpr (C::kQ4) {
+              beta = fmaf(wgt[j], fmaf(1.5f, s, mn), beta);
+              axpy16<false>(acc, wgt[j] * s * pow2i(87), vh, 0u);
+            } else {
+              beta = fmaf(wgt[j], mn, beta);
+              axpy16<false>(acc, wgt[j] * s * pow2i(85), vh, 0u);
+            }
+          } else {
+            const uint4* vp = reinterpret_cast<const uint4*>(st + (t >> 4) * LOAD + R::kBfV + (t & 15) * D * 2 + 32 * k);
+            const uint4 a = vp[0], c = vp[1];
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+            const float2 ww = make_float2(wgt[j], wgt[j]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __ffma2_rn(ww, make_float2(bf16_lo(w[i]), bf16_hi(w[i])), acc[i]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar + 8 * stage);
+      }
+    }
+  }
+
+  // ---- warp results: true per-channel sums, reduced over token sub-groups
+  if (warp < kNW) {
+    float o[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if constexpr (C::kQuant) {
+        const int pa = (C::kQ4 && FULLV) ? pos4(2 * i) : pos2(2 * i);
+        const int pb = (C::kQ4 && FULLV) ? pos4(2 * i + 1) : pos2(2 * i + 1);
+        o[2 * i] = fmaf(acc[i].x, pow2i(64 - pa), beta);
+        o[2 * i + 1] = fmaf(acc[i].y, pow2i(64 - pb), beta);
+      } else {
+        o[2 * i] = acc[i].x;
+        o[2 * i + 1] = acc[i].y;
+      }
+    }
+#pragma unroll
+    for (int off = CH; off < 32; off <<= 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) o[i] += __shfl_xor_sync(0xffffffffu, o[i], off);
+      l_w += __shfl_xor_sync(0xffffffffu, l_w, off);
+    }
+    float* ws = wscr + warp * (D + 4);
+    if (r == 0) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) ws[16 * k + i] = o[i];
+    }
+    if (lane == 0) {
+      ws[D] = m_w;
+      ws[D + 1] = l_w;
+    }
+  }
+  __syncthreads();
+  // ---- CTA merge (CTA-local scale m_cta)
+  {
+    float m_c = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kNW; ++w) m_c = fmaxf(m_c, wscr[w * (D + 4) + D]);
+    if (threadIdx.x < D) {
+      float a = 0.f;
+#pragma unroll
+      for (int w = 0; w < kNW; ++w) {
+        const float mw = wscr[w * (D + 4) + D];
+        if (mw != -INFINITY) a = fmaf(fast_exp2(mw - m_c), wscr[w * (D + 4) + threadIdx.x], a);
+      }
+      cta_acc[threadIdx.x] = a;
+    }
+    if (threadIdx.x == 0) {
+      float l = 0.f;
+#pragma unroll
+      for (int w = 0; w < kNW; ++w) {
+        const float mw = wscr[w * (D + 4) + D];
+        if (mw != -INFINITY) l = fmaf(fast_exp2(mw - m_c), wscr[w * (D + 4) + D + 1], l);
+      }
+      cta_f[kSlotM] = m_c;
+      cta_f[kSlotL] = l;
+    }
+  }
+  if constexpr (CLUSTER) cluster_sync_all(); else __syncthreads();
+
+  // ---- global (max, normaliser) over the splits
+  float m_g = -INFINITY, z = 0.f;
+  int any_bad = 0;
+  const uint32_t my_f = smem_addr(cta_f);
+  for (int s = 0; s < S; ++s) {
+    float ms, ls;
+    int bs;
+    if constexpr (CLUSTER) {
+      const uint32_t pa = peer_addr(my_f, s);
+      ms = ld_peer_f32(pa + 4 * kSlotM);
+      ls = ld_peer_f32(pa + 4 * kSlotL);
+      bs = ld_peer_s32(pa + 4 * kSlotBad);
+    } else {
+      ms = cta_f[kSlotM];
+      ls = cta_f[kSlotL];
+      bs = cta_i[kSlotBad];
+    }
+    any_bad |= bs;
+    if (ms != -INFINITY) {
+      if (ms > m_g) {
+        z = z * fast_exp2(m_g - ms) + ls;
+        m_g = ms;
+      } else {
+        z = fmaf(ls, fast_exp2(ms - m_g), z);
+      }
+    }
+  }
+  const bool live = !any_bad && z > 0.f;
+  const float inv_z = live ? 1.f / z : 0.f;
+
+  // ---- pass 2: low-plane selection and gather (4-bit sources)
+  pdl_wait_prior_grid();  // nothing below writes memory the previous kernel may still use
+  const bool want_mask = p.sel_mask != nullptr || p.sel_count != nullptr;
+  if (warp < kNW && live && ((C::kLogits && p.tau < INFINITY) || want_mask)) {
+    const float m_c = cta_f[kSlotM];
+    float corr[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) corr[i] = 0.f;
+    int cnt = 0;
+    for (int gi = warp; gi < cg; gi += kNW) {
+      const bool valid = (g0 + gi) * kGroup + lane < nn;
+      float lg = 0.f;
+      bool sel;
+      if constexpr (C::kLogits) {
+        lg = logits[gi * kGroup + lane];
+        sel = valid && (fast_exp2(lg - m_g) * inv_z >= p.tau);
+      } else {
+        sel = C::kQ4 && valid;  // tau = 0: every token took its low plane in pass 1
+      }
+      const uint32_t mask = __ballot_sync(0xffffffffu, sel);
+      if (p.sel_mask && lane == 0)
+        p.sel_mask[(static_cast<size_t>(b) * p.H + h) * p.mask_words + g0 + gi] = mask;
+      cnt += __popc(mask);
+      if constexpr (C::kLogits) {
+        const int nsel = __popc(mask);
+        for (int base = 0; base < nsel; base += TS) {
+          const int my = base + r;
+          uint32_t mm = mask;
+          for (int q = 0; q < my && mm; ++q) mm &= mm - 1;
+          const int t = (my < nsel) ? (__ffs(mm) - 1) : 0;
+          const float lt = __shfl_sync(0xffffffffu, lg, t);
+          if (my < nsel) {
+            const int phys = ids[2 * gi + (t >> 4)];
+            const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
+            const uint32_t lo = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VLo + (t & 15) * R::kRow + 4 * k);
+            const uint32_t mv = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VMeta + ((t & 15) * (D / kGroup) + (k >> 1)) * 4);
+            const float ws = fast_exp2(lt - m_c) * bf16_lo(mv);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              corr[i] = fmaf(ws, static_cast<float>((lo >> (2 * i)) & 3u) - 1.5f, corr[i]);
+          }
+        }
+      }
+    }
+    if constexpr (C::kLogits) {
+#pragma unroll
+      for (int off = CH; off < 32; off <<= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) corr[i] += __shfl_xor_sync(0xffffffffu, corr[i], off);
+      if (r == 0) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) atomicAdd(&cta_acc[16 * k + i], corr[i]);
+      }
+    }
+    if (lane == 0) atomicAdd(&cta_i[kSlotCount], cnt);
+  }
+  if constexpr (CLUSTER) cluster_sync_all(); else __syncthreads();
+
+  // ---- combine the splits; rank s writes channels [s*D/S, (s+1)*D/S)
+  const int per_rank = D / S;
+  if (threadIdx.x < per_rank) {
+    const int c = split * per_rank + threadIdx.x;
+    float v = 0.f;
+    if (live) {
+      for (int s = 0; s < S; ++s) {
+        float ms, as;
+        if constexpr (CLUSTER) {
+          const uint32_t pa = peer_addr(my_f, s);
+          ms = ld_peer_f32(pa + 4 * kSlotM);
+          as = ld_peer_f32(peer_addr(smem_addr(cta_acc + c), s));
+        } else {
+          ms = cta_f[kSlotM];
+          as = cta_acc[c];
+        }
+        if (ms != -INFINITY) v = fmaf(as, fast_exp2(ms - m_g), v);
+      }
+      v *= inv_z;
+    }
+    p.out[(static_cast<size_t>(b) * p.H + h) * D + c] = __float2bfloat16_rn(v);
+  }
+  if (split == 0 && threadIdx.x == 0) {
+    if (p.sel_count) {
+      int total = 0;
+      if (live && (C::kQ4)) {
+        for (int s = 0; s < S; ++s) {
+          if constexpr (CLUSTER) total += ld_peer_s32(peer_addr(smem_addr(&cta_i[kSlotCount]), s));
+          else total += cta_i[kSlotCount];
+        }
+      }
+      p.sel_count[static_cast<size_t>(b) * p.H + h] = total;
+    }
+    if (any_bad) flag_error(p.err, any_bad);
+  }
+  if constexpr (CLUSTER) cluster_sync_all();  // peers' shared memory stays alive until here
+}
+
+template <int KIND, int D, bool FULLV, bool CLUSTER>
+cudaError_t launch_t(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
+  using C = Cfg<KIND, D, FULLV>;
+  const Smem sp = smem_plan(C::kStage, C::kNS, p.chunk_groups, D, C::kLogits);
+  if (sp.total > 227u * 1024u) return cudaErrorInvalidValue;
+  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sp.total));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(splits, p.H, batch);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = sp.total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (CLUSTER) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = splits;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int KIND, int D, bool FULLV>
+cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
+  return splits > 1 ? launch_t<KIND, D, FULLV, true>(p, batch, splits, stream, pdl)
+                    : launch_t<KIND, D, FULLV, false>(p, batch, splits, stream, pdl);
+}
+
+}  // namespace
+
+namespace {
+size_t smem_for(int kind, int head_dim, bool full_values, int cg) {
+  int rec, load, ns = 8;
+  const int plane = 16 * head_dim / 4, kmeta = head_dim * 2, vmeta = 16 * (head_dim / 32) * 4;
+  if (kind == LOOPKV_CELL_Q4) {
+    rec = 4 * plane + kmeta + vmeta;
+    load = full_values ? rec : rec - plane;
+  } else if (kind == LOOPKV_CELL_Q2) {
+    load = 2 * plane + kmeta + vmeta;
+  } else {
+    load = 64 * head_dim;
+    ns = 4;
+  }
+  return smem_plan(2 * load, ns, cg, head_dim, kind == LOOPKV_CELL_Q4 && !full_values).total;
+}
+}  // namespace
+
+// Largest context one split may hold (its logits live in shared memory).
+constexpr int kMaxGroupsPerSplit = 512;
+
+int decode_splits(int kind, int head_dim, int batch, int heads, int max_seq_len) {
+  const int groups = (max_seq_len + kGroup - 1) / kGroup;
+  const long pairs = static_cast<long>(batch) * heads;
+  int min_s = 1;
+  while (min_s < 8 && (groups + min_s - 1) / min_s > kMaxGroupsPerSplit) min_s <<= 1;
+  if (pairs <= 0 || groups <= 1) return min_s;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int best = min_s;
+  double best_eff = -1.0;
+  for (int s = min_s; s <= 8; s <<= 1) {
+    if (s > min_s && groups < 4 * s) break;  // keep at least 4 groups per split
+    const int cg = (groups + s - 1) / s;
+    const size_t smem = smem_for(kind, head_dim, false, cg) + 1024;
+    const long per_sm = std::min<long>(4, static_cast<long>((228u * 1024u) / smem));
+    const long slots = static_cast<long>(sms) * std::max<long>(1, per_sm);
+    const long ctas = pairs * s;
+    const long waves = (ctas + slots - 1) / slots;
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
+
+cudaError_t launch_decode(int kind, int head_dim, const DecodeParams& p, int batch, int splits,
+                          bool full_values, cudaStream_t stream, bool pdl) {
+  if (batch == 0) return cudaSuccess;
+  const int key = kind * 1000 + head_dim;
+  switch (key) {
+    case LOOPKV_CELL_Q4 * 1000 + 128:
+      return full_values ? launch_c<LOOPKV_CELL_Q4, 128, true>(p, batch, splits, stream, pdl)
+                         : launch_c<LOOPKV_CELL_Q4, 128, false>(p, batch, splits, stream, pdl);
+    case LOOPKV_CELL_Q4 * 1000 + 64:
+      return full_values ? launch_c<LOOPKV_CELL_Q4, 64, true>(p, batch, splits, stream, pdl)
+                         : launch_c<LOOPKV_CELL_Q4, 64, false>(p, batch, splits, stream, pdl);
+    case LOOPKV_CELL_Q2 * 1000 + 128: return launch_c<LOOPKV_CELL_Q2, 128, false>(p, batch, splits, stream, pdl);
+    case LOOPKV_CELL_Q2 * 1000 + 64: return launch_c<LOOPKV_CELL_Q2, 64, false>(p, batch, splits, stream, pdl);
+    case LOOPKV_CELL_BF16 * 1000 + 128: return launch_c<LOOPKV_CELL_BF16, 128, false>(p, batch, splits, stream, pdl);
+    case LOOPKV_CELL_BF16 * 1000 + 64: return launch_c<LOOPKV_CELL_BF16, 64, false>(p, batch, splits, stream, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace loopkv

@@ -364,28 +364,3 @@ def unpack_plane(plane_bytes, d: int) -> np.ndarray:
     for i in range(4):
         out[:, i::4] = (b >> (2 * i)) & 3
     return out
-
-
-# ---------------------------------------------------------------------------
-# Algorithmic bytes (what one decode launch must read and write)
-# ---------------------------------------------------------------------------
-
-def decode_bytes(kind: str, d: int, n: int, n_selected: int, block: int = BLOCK) -> int:
-    """Bytes one (cell, sequence, head) decode must move: K and V at the cell's
-    precision (4-bit values: high plane for every token, low plane for the
-    selected ones), the exact key tail, the block-table entries, the query and
-    the output."""
-    q_out = 2 * d * 2 + 4 * (-(-n // block))
-    if n == 0:
-        return q_out
-    if kind == "bf16":
-        return q_out + n * 4 * d
-    ng = n // GROUP
-    full = ng * GROUP
-    plane = d // 4
-    k_meta = ng * d * 4
-    tail = (n - full) * d * 2
-    v_meta = n * (d // GROUP) * 4
-    if kind == "q4":
-        return q_out + full * 2 * plane + k_meta + tail + n * plane + v_meta + n_selected * plane
-    return q_out + full * plane + k_meta + tail + n * plane + v_meta

@@ -1,0 +1,121 @@
+"""Shared helpers of the GPU parity tests: build cells through the C ABI on
+seeded inputs and compare them, output by output, with the CPU oracle."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle as O
+from workload import block_table_for, cell_kv, cell_query, make_plan, seq_lens_for
+
+# Output tolerance of the attention result: |gpu - oracle| <= ATOL + RTOL*|oracle|
+ATOL, RTOL = 2e-3, 1e-2
+# Selection may differ only where the oracle's weight is this close to tau
+SEL_WINDOW = 1e-6
+
+
+def build_store(w, cells=None, capacity=None, device="cuda", flags=0, splits=0, prefill=True):
+    """Allocate the cells of workload ``w`` and bulk-append its seeded K/V.
+
+    ``cells`` limits which cells get storage and data (reuse cells always
+    need their final-loop source).  Returns (kv, plan, table, lens, kvdata)
+    with kvdata[cell] = (K, V) bf16 [B, n_max, H, D] on the device.
+    """
+    from mixed_precision_kv_loopkv_b200 import KVCells, loopkv_quantize_append
+
+    plan = make_plan(w)
+    lens = seq_lens_for(w)
+    cap = lens if capacity is None else capacity
+    table, num_blocks = block_table_for(w, cap)
+    want = set(range(len(plan))) if cells is None else set(cells)
+    for c in list(want):
+        if plan[c] == "reuse":
+            want.add((w.num_loops - 1) * w.num_layers + c % w.num_layers)
+    kv = KVCells(plan, w.num_loops, w.num_layers, w.num_heads, w.head_dim, num_blocks,
+                 w.batch, table.shape[1], device=device, flags=flags, decode_splits=splits,
+                 allocate=want)
+    table_d = torch.from_numpy(table).to(device)
+    lens_d = torch.from_numpy(lens).to(device)
+    zero = torch.zeros(w.batch, dtype=torch.int32, device=device)
+    data = {}
+    if prefill:
+        for c in sorted(want):
+            if plan[c] == "reuse":
+                continue
+            loop, layer = divmod(c, w.num_layers)
+            k, v = cell_kv(w, loop, layer, device=device)
+            loopkv_quantize_append(kv, loop, layer, k, v, table_d, zero)
+            data[c] = (k, v)
+    return kv, plan, table_d, lens_d, data
+
+
+def oracle_pair(kind, k, v, q, tau, sm_scale):
+    """Oracle decode of one (cell, sequence, head) from bf16 tensors."""
+    seq = O.StoredSequence(kind, k.float().cpu().numpy(), v.float().cpu().numpy())
+    return seq.attend(q.float().cpu().numpy(), tau, sm_scale)
+
+
+def unpack_mask(words: torch.Tensor, n: int) -> np.ndarray:
+    w = words.cpu().numpy().astype(np.int64) & 0xFFFFFFFF
+    bits = ((w[:, None] >> np.arange(32)) & 1).astype(bool).reshape(-1)
+    return bits[:n]
+
+
+def check_cell(kv, plan, cell, data, q, table, lens, tau, sm_scale, pairs, out=None,
+               sel_mask=None, sel_count=None, report=None):
+    """Compare one decoded cell with the oracle on the given (b, h) pairs."""
+    src = kv.source_cell(cell)
+    kind = plan[src]
+    k_all, v_all = data[src]
+    lens_h = lens.cpu().numpy()
+    out_h = out.float().cpu()
+    worst = 0.0
+    mism = 0
+    for (b, h) in pairs:
+        n = int(lens_h[b])
+        o, sel, p = oracle_pair(kind, k_all[b, :n, h], v_all[b, :n, h], q[b, h], tau, sm_scale)
+        got = out_h[b, h].numpy().astype(np.float64)
+        err = np.abs(got - o) - (ATOL + RTOL * np.abs(o))
+        worst = max(worst, float(np.max(np.abs(got - o))) if n else 0.0)
+        if np.any(err > 0):
+            i = int(np.argmax(err))
+            raise AssertionError(f"cell {cell} ({kind}) b={b} h={h} n={n}: channel {i} "
+                                 f"gpu {got[i]:.6g} oracle {o[i]:.6g}")
+        if sel_mask is not None and n:
+            g = unpack_mask(sel_mask[b, h], n)
+            diff = np.nonzero(g != sel)[0]
+            bad = [t for t in diff if abs(p[t] - tau) >= SEL_WINDOW]
+            if bad:
+                t = bad[0]
+                raise AssertionError(f"cell {cell} b={b} h={h}: token {t} selected gpu={g[t]} "
+                                     f"oracle={sel[t]} p={p[t]:.9g} tau={tau}")
+            mism += len(diff)
+        if sel_count is not None:
+            want = int(sel.sum())
+            got_c = int(sel_count[b, h])
+            if sel_mask is not None:
+                want = int(unpack_mask(sel_mask[b, h], n).sum()) if n else 0
+            assert got_c == want, (cell, b, h, got_c, want)
+    if report is not None:
+        report.append({"cell": cell, "kind": kind, "max_abs_err": worst, "sel_mismatch_in_window": mism})
+    return worst, mism
+
+
+def query_for(w, cell, device="cuda", temperature=None):
+    loop, layer = divmod(cell, w.num_layers)
+    return cell_query(w, loop, layer, device=device, temperature=temperature)
+
+
+def sample_pairs(w, nseq, seed=0):
+    rng = np.random.default_rng(seed)
+    seqs = sorted(rng.choice(w.batch, size=min(nseq, w.batch), replace=False).tolist())
+    return [(b, h) for b in seqs for h in range(w.num_heads)]
+
+
+def mask_buffers(kv, batch, device="cuda"):
+    words = math.ceil(kv.max_blocks_per_seq * kv.block_size / 32)
+    return (torch.zeros((batch, kv.num_heads, words), dtype=torch.int32, device=device),
+            torch.zeros((batch, kv.num_heads), dtype=torch.int32, device=device))

@@ -1,0 +1,28 @@
+"""Byte accounting of the benchmark (host logic, no GPU)."""
+
+from mixed_precision_kv_loopkv_b200.accounting import decode_bytes, step_bytes
+
+
+def test_per_token_head_bytes():
+    """4-bit: 128 bytes per token-head plus 32 per selected token (D = 128);
+    2-bit: 96; bf16: 512; plus query, output and block-table entries."""
+    fixed = 2 * 128 * 2 + 4 * (4096 // 16)
+    assert decode_bytes("q4", 128, 4096, 0) - fixed == 128 * 4096
+    assert decode_bytes("q4", 128, 4096, 100) - fixed == 128 * 4096 + 32 * 100
+    assert decode_bytes("q2", 128, 4096, 0) - fixed == 96 * 4096
+    assert decode_bytes("bf16", 128, 4096, 0) - fixed == 512 * 4096
+    assert decode_bytes("q4", 64, 0, 0) == 256
+
+
+def test_unfinished_key_group_reads_exact_tail():
+    # 40 tokens: one quantised key group (32) + 8 exact bf16 keys
+    got = decode_bytes("q2", 128, 40)
+    want = 512 + 4 * 3 + 32 * 32 + 32 * 128 * 4 // 32 + 8 * 256 + 40 * 32 + 40 * 16
+    assert got == want
+
+
+def test_step_bytes_resolves_reuse():
+    plan = ["reuse", "q2", "q4", "q4"]          # 2 loops x 2 layers
+    b1 = step_bytes(plan, 2, 2, 128, 1, [64], [64])
+    want = 2 * decode_bytes("q4", 128, 64) + decode_bytes("q2", 128, 64) + decode_bytes("q4", 128, 64)
+    assert b1 == want

@@ -1,0 +1,69 @@
+"""Host logic of bench.py on CPU: the slowest-rank reduction and the
+whole-job aggregate over world_size 2 gloo ranks, plus the reference arm's
+bookkeeping."""
+
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    bench.init_dist(world, rank, backend="gloo")
+    ms = [12.5, 20.0][rank]
+    slowest = bench.max_over_ranks(ms, world)
+    bench.barrier(world)
+    value = bench.aggregate_value(1e9, world, slowest / 1e3)
+    q.put((rank, slowest, value))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_two_rank_max_and_aggregate():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, slowest, value in res:
+        assert slowest == 20.0
+        assert value == pytest.approx(2 * 1e9 / 0.020 / 1e9)
+
+
+def test_single_rank_helpers():
+    assert bench.max_over_ranks(3.0, 1) == 3.0
+    assert bench.aggregate_value(2e9, 1, 1.0) == 2.0
+
+
+def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "decode_attention_demo.md").write_text(
+        f"- source_sha256: `{bench.decode_source_hash()}`\n- dram_bytes_per_launch: 1234\n")
+    csrc = tmp_path / "mixed_precision_kv_loopkv_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("decode.cu", "device_common.cuh"):
+        src = os.path.join(bench.ROOT, "mixed_precision_kv_loopkv_b200", "csrc", f)
+        (csrc / f).write_bytes(open(src, "rb").read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("demo") == 1234.0
+    (csrc / "decode.cu").write_text("// changed\n")
+    assert bench.profiled_traffic("demo") is None

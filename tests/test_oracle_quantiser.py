@@ -232,13 +232,3 @@ def test_bf16_records_are_raw_rows():
     assert resid is None and rec.shape == (2, O.record_bytes("bf16", 64))
     kr = rec[1, : 16 * 128].copy().view("<u2").reshape(16, 64)
     np.testing.assert_array_equal(kr[3], torch.from_numpy(k[19]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
-
-
-def test_decode_bytes_per_token_head():
-    """4-bit: 128 bytes per token-head plus 32 per selected token (d = 128);
-    2-bit: 96; bf16: 512; plus query, output and block-table entries."""
-    fixed = 2 * 128 * 2 + 4 * (4096 // 16)
-    assert O.decode_bytes("q4", 128, 4096, 0) - fixed == 128 * 4096
-    assert O.decode_bytes("q4", 128, 4096, 100) - fixed == 128 * 4096 + 32 * 100
-    assert O.decode_bytes("q2", 128, 4096, 0) - fixed == 96 * 4096
-    assert O.decode_bytes("bf16", 128, 4096, 0) - fixed == 512 * 4096
