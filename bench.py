@@ -52,6 +52,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (a smaller case of the same kernel)")
+    ap.add_argument("--cells", type=int, default=0,
+                    help="run only the first N cells (and their reuse sources): a small case for ncu")
     return ap.parse_args(argv)
 
 
@@ -192,7 +196,7 @@ def profiled_traffic(workload: str):
 
 # ----------------------------------------------------------------- workload setup
 
-def setup(w, pdl: bool, splits: int, extra: int = 64):
+def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0):
     from mixed_precision_kv_loopkv_b200 import (LOOPKV_FLAG_PDL, KVCells, LoopedDecodeStep,
                                                 loopkv_quantize_append)
     from workload import block_table_for, cell_kv, cell_new_token, cell_query, make_plan, seq_lens_for
@@ -200,17 +204,22 @@ def setup(w, pdl: bool, splits: int, extra: int = 64):
     plan = make_plan(w)
     lens = seq_lens_for(w)
     table_np, num_blocks = block_table_for(w, lens + extra)
+    C = len(plan)
+    run = list(range(C))
+    if ncells:
+        src = lambda c: c if plan[c] != "reuse" else (w.num_loops - 1) * w.num_layers + c % w.num_layers
+        run = sorted(set(range(ncells)) | {src(c) for c in range(ncells)})
     kv = KVCells(plan, w.num_loops, w.num_layers, w.num_heads, w.head_dim, num_blocks, w.batch,
-                 table_np.shape[1], flags=LOOPKV_FLAG_PDL if pdl else 0, decode_splits=splits)
+                 table_np.shape[1], flags=LOOPKV_FLAG_PDL if pdl else 0, decode_splits=splits,
+                 allocate=set(run))
     table = torch.from_numpy(table_np).cuda()
     zero = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
-    stored = [c for c, k in enumerate(plan) if k != "reuse"]
+    stored = [c for c in run if plan[c] != "reuse"]
     for c in stored:
         loop, layer = divmod(c, w.num_layers)
         k, v = cell_kv(w, loop, layer, device="cuda")
         loopkv_quantize_append(kv, loop, layer, k, v, table, zero)
         del k, v
-    C = len(plan)
     q_all = torch.stack([cell_query(w, *divmod(c, w.num_layers), device="cuda") for c in range(C)])
     kn_all = torch.empty((len(stored), w.batch, 1, w.num_heads, w.head_dim), dtype=torch.bfloat16,
                          device="cuda")
@@ -225,7 +234,7 @@ def setup(w, pdl: bool, splits: int, extra: int = 64):
         kv, table, pos, [q_all[c] for c in range(C)],
         {c: kn_all[slot[c]] for c in stored}, {c: vn_all[slot[c]] for c in stored},
         [out_all[c] for c in range(C)], w.tau, w.sm_scale, int(lens.max()) + 1,
-        sel_count=[sel_all[c] for c in range(C)])
+        sel_count=[sel_all[c] for c in range(C)], cells=run)
     torch.cuda.synchronize()
     return dict(plan=plan, lens=lens, kv=kv, step=step, q_all=q_all, kn_all=kn_all, vn_all=vn_all,
                 out_all=out_all, sel_all=sel_all)
@@ -370,7 +379,9 @@ def main_arm(args, world, rank, local):
     torch.cuda.set_device(local)
     init_dist(world, local)
     w = get_workload(args.workload)
-    S = setup(w, pdl=not args.no_pdl, splits=args.splits)
+    if args.batch:
+        w = w.with_(batch=args.batch)
+    S = setup(w, pdl=not args.no_pdl, splits=args.splits, ncells=args.cells)
     step, plan, lens = S["step"], S["plan"], S["lens"]
     dev = torch.device(f"cuda:{local}")
 
@@ -385,7 +396,8 @@ def main_arm(args, world, rank, local):
     ms_max = max_over_ranks(ms, world, dev)
 
     sel = S["sel_all"].cpu().numpy()
-    bytes_step = step_bytes(plan, w.num_layers, w.num_loops, w.head_dim, w.num_heads, lens + 1, lens, sel)
+    bytes_step = step_bytes(plan, w.num_layers, w.num_loops, w.head_dim, w.num_heads, lens + 1, lens, sel,
+                            cells=step.cells)
     value = aggregate_value(bytes_step * args.steps, world, ms_max / 1e3)
     us_step = ms_max / args.steps * 1e3
 
@@ -433,6 +445,8 @@ def main_arm(args, world, rank, local):
 
     if rank == 0:
         cfg = workload_config(w, world)
+        if args.cells:
+            cfg["cells_run"] = len(step.cells)
         cfg.update({"pdl": not args.no_pdl, "splits": args.splits or "auto", "cuda_graph": True,
                     "algorithmic_bytes_per_step": bytes_step,
                     "selected_low_plane_rows_per_step": int(sel.sum())})

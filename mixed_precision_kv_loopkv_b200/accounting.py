@@ -38,12 +38,14 @@ def decode_bytes(kind: str, d: int, n: int, n_selected: int = 0) -> int:
 
 
 def step_bytes(plan, num_layers: int, num_loops: int, d: int, heads: int, lens_stored, lens_reuse,
-               selected=None) -> int:
+               selected=None, cells=None) -> int:
     """Bytes of one looped decode step: every cell decodes every (sequence,
     head); stored cells over lens_stored[b] tokens, reuse cells over the
     final loop's lens_reuse[b]; selected[cell][b][h] low-plane rows."""
     total = 0
     for cell, kind in enumerate(plan):
+        if cells is not None and cell not in cells:
+            continue
         src = cell if kind != "reuse" else (num_loops - 1) * num_layers + cell % num_layers
         src_kind = plan[src]
         lens = lens_reuse if kind == "reuse" else lens_stored

@@ -10,14 +10,14 @@
 // streaming-softmax idea (O(1)-memory attention in the same pages' listing).
 //
 // Grid (splits, heads, batch); the splits of one (sequence, head) form one
-// thread-block cluster.  Each CTA:
-//   - a producer lane streams the pass-1 prefix of every block record of its
-//     context chunk (keys, key meta, value high plane, value meta: 2048 B of
-//     the 2560-B 4-bit record at D = 128) with 1-D bulk copies (TMA, no
-//     multicast) into an NS-stage shared-memory ring;
-//   - NW consumer warps each take whole 32-token groups: dequantise the keys
-//     at the cell's precision, form the logits, keep an online softmax and
-//     accumulate the high-plane values;
+// thread-block cluster.  Each CTA owns a chunk of 32-token groups:
+//   - every warp streams its own groups (interleaved with the other warps)
+//     through a private ring of shared-memory stages: lane 0 issues 1-D bulk
+//     copies (TMA, no multicast) of each block record's pass-1 prefix (keys,
+//     key meta, value high plane, value meta: 2048 B of the 2560-B 4-bit
+//     record at D = 128), completion on an mbarrier per stage;
+//   - the warp dequantises the keys at the cell's precision, forms the
+//     logits, keeps an online softmax and accumulates the high-plane values;
 //   - the splits exchange (max, sum) through distributed shared memory, so
 //     every CTA knows the exact normaliser Z before any low-plane read;
 //   - pass 2 re-reads the CTA's logits from shared memory, ballots the tokens
@@ -42,18 +42,18 @@
 namespace loopkv {
 namespace {
 
-constexpr int kNW = 4;        // consumer warps per CTA
-constexpr int kThreads = 32 * (kNW + 1);
-constexpr int kExpOff = 64;   // E: products live at 2^-64 of their true size
+constexpr int kNW = 4;                 // warps per CTA, each streams its own groups
+constexpr int kThreads = 32 * kNW;
+constexpr int kExpOff = 64;            // E: key products live at 2^-64 of their size
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 
 // Field position (bits) of channel i of a 16-channel chunk.
 // 2-bit plane word: channel i at bits 2i; i >= 11 is read from (w >> 22).
-__device__ __forceinline__ constexpr int pos2(int i) { return 2 * (i < 11 ? i : i - 11); }
+__host__ __device__ constexpr int pos2(int i) { return 2 * (i < 11 ? i : i - 11); }
 // 4-bit nibble words (even/odd channels): channel i in nibble i/2;
 // nibbles >= 5 are read from (w >> 20).
-__device__ __forceinline__ constexpr int pos4(int i) { return 4 * ((i >> 1) < 5 ? (i >> 1) : (i >> 1) - 5); }
+__host__ __device__ constexpr int pos4(int i) { return 4 * ((i >> 1) < 5 ? (i >> 1) : (i >> 1) - 5); }
 
 // Subnormal view of field i of a 2-bit plane word.
 __device__ __forceinline__ float fld2(uint32_t w, uint32_t w22, int i) {
@@ -70,28 +70,27 @@ __device__ __forceinline__ void combine_planes(uint32_t hi, uint32_t lo, uint32_
   odd = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
 }
 
-// Dot product of 16 subnormal code views with 16 pre-scaled coefficients.
+// Dot product of 16 subnormal code views with 16 pre-scaled coefficients
+// (pairs of channels 2p, 2p+1).
 template <bool FOUR>
-__device__ __forceinline__ float dot16(const float* c, uint32_t a, uint32_t b, float init) {
+__device__ __forceinline__ float dot16(const float2* c, uint32_t a, uint32_t b, float init) {
   float2 acc = make_float2(init, 0.f);
-  if constexpr (FOUR) {  // a, b = even/odd nibble words
+  if constexpr (FOUR) {  // a, b = high / low plane words
     uint32_t e, o;
     combine_planes(a, b, e, o);
     const uint32_t e20 = e >> 20, o20 = o >> 20;
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
-      acc = __ffma2_rn(make_float2(c[2 * m], c[2 * m + 1]), make_float2(nib(e, e20, m), nib(o, o20, m)), acc);
+    for (int m = 0; m < 8; ++m) acc = __ffma2_rn(c[m], make_float2(nib(e, e20, m), nib(o, o20, m)), acc);
   } else {  // a = 2-bit plane word
     const uint32_t a22 = a >> 22;
 #pragma unroll
     for (int p = 0; p < 8; ++p)
-      acc = __ffma2_rn(make_float2(c[2 * p], c[2 * p + 1]),
-                       make_float2(fld2(a, a22, 2 * p), fld2(a, a22, 2 * p + 1)), acc);
+      acc = __ffma2_rn(c[p], make_float2(fld2(a, a22, 2 * p), fld2(a, a22, 2 * p + 1)), acc);
   }
   return acc.x + acc.y;
 }
 
-// acc[p] += w * (codes 2p, 2p+1)
+// acc[p] += w * (codes of channels 2p, 2p+1)
 template <bool FOUR>
 __device__ __forceinline__ void axpy16(float2* acc, float w, uint32_t a, uint32_t b) {
   const float2 ww = make_float2(w, w);
@@ -117,24 +116,26 @@ struct Cfg {
   // bytes of one block record streamed in pass 1
   static constexpr int kLoad = kQ4 ? (FULLV ? R::kBytes : R::kQ4VLo) : R::kBytes;
   static constexpr int kStage = 2 * kLoad;                 // one 32-token group
-  static constexpr int kNS = kQuant ? 8 : 4;               // ring stages
+  static constexpr int kNSW = kQuant ? 3 : 2;              // ring stages per warp
   static constexpr int kCH = D / 16;                       // lanes per token
   static constexpr int kTS = 32 / kCH;                     // token sub-groups per warp
   static constexpr int kTPL = kCH;                         // tokens per lane per group
   static constexpr int kE = kQuant ? kExpOff : 0;
+  // power of two folded into the softmax weight for the value products
+  static constexpr int kVSh = !kQuant ? 0 : (kQ4 && !FULLV) ? 87 : 85;
   static constexpr bool kLogits = kQ4 && !FULLV;           // pass 2 needs the logits
+  static constexpr bool kFourV = kQ4 && FULLV;             // full 4-bit values in pass 1
 };
 
 // Shared-memory carve-up (bytes), identical on host and device.
 struct Smem {
-  size_t stages, bars, ids, logits, wscr, cta, total;
+  size_t rings, bars, logits, wscr, cta, total;
 };
-__host__ __device__ inline Smem smem_plan(int stage_bytes, int ns, int cg, int d, bool logits) {
+__host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int d, bool logits) {
   Smem s;
-  s.stages = 0;
-  s.bars = s.stages + static_cast<size_t>(stage_bytes) * ns;
-  s.ids = s.bars + 16 * ns;
-  s.logits = s.ids + ((8 * cg + 15) / 16) * 16;
+  s.rings = 0;
+  s.bars = s.rings + static_cast<size_t>(stage_bytes) * nsw * kNW;
+  s.logits = s.bars + 8 * nsw * kNW;
   s.wscr = s.logits + (logits ? 128 * static_cast<size_t>(cg) : 0);
   s.cta = s.wscr + static_cast<size_t>(kNW) * (d + 4) * 4;
   s.total = s.cta + static_cast<size_t>(d + 4) * 4;
@@ -144,19 +145,172 @@ __host__ __device__ inline Smem smem_plan(int stage_bytes, int ns, int cg, int d
 // Per-CTA scalar slots in the cta segment after the D accumulators.
 enum { kSlotM = 0, kSlotL = 1, kSlotCount = 2, kSlotBad = 3 };
 
-template <int KIND, int D, bool FULLV, bool CLUSTER>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
+// Per-lane running state of one warp's online softmax.
+struct WarpState {
+  float m, l, beta;
+  float2 acc[8];
+};
+
+// One 32-token group.  Lane (r, k): channels 16k..16k+15 of tokens
+// r + TS*j (j < TPL).  TAIL: the sequence's unfinished key group, keys from
+// the exact residual and tokens past the end masked.
+template <int KIND, int D, bool FULLV, bool TAIL>
+__device__ __forceinline__ void group_step(const uint8_t* st, const float* qf, const float* qs,
+                                           const __nv_bfloat16* res, int tok0, int nn, int r, int k,
+                                           float* logits_g, WarpState& ws) {
   using C = Cfg<KIND, D, FULLV>;
   using R = typename C::R;
-  constexpr int CH = C::kCH, TS = C::kTS, TPL = C::kTPL, NS = C::kNS;
+  constexpr int CH = C::kCH, TS = C::kTS, TPL = C::kTPL, LOAD = C::kLoad;
+  const float esc = pow2i(C::kE);
+
+  // this lane's row word of token j: rowbase + offset(j), a compile-time offset
+  const uint8_t* rowbase = st + r * R::kRow + 4 * k;
+  auto tok_off = [](int j) { return ((TS * j) >> 4) * LOAD + ((TS * j) & 15) * R::kRow; };
+
+  // ---- keys -> logits (scaled by 2^-E)
+  float part[TPL];
+  if constexpr (C::kQuant && !TAIL) {
+    const uint8_t* km = st + ((16 * k < D / 2) ? 0 : LOAD) + R::kKMetaOff + ((16 * k) % (D / 2)) * 4;
+    float2 q2[8];
+    float2 al = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 mw = reinterpret_cast<const uint4*>(km)[v];
+      const uint32_t w4[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int i = 4 * v + 2 * u;
+        q2[i / 2] = __fmul2_rn(make_float2(qs[i], qs[i + 1]),
+                               make_float2(bf16_lo(w4[2 * u]), bf16_lo(w4[2 * u + 1])));
+        al = __ffma2_rn(make_float2(qf[i], qf[i + 1]),
+                        make_float2(bf16_hi(w4[2 * u]), bf16_hi(w4[2 * u + 1])), al);
+      }
+    }
+    const float alpha = (al.x + al.y) * pow2i(-C::kE);
+#pragma unroll
+    for (int j = 0; j < TPL; ++j) {
+      const uint8_t* row = rowbase + tok_off(j);
+      const uint32_t w0 = *reinterpret_cast<const uint32_t*>(row + R::kKHi);
+      if constexpr (C::kQ4) {
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(row + R::kQ4KLo);
+        part[j] = dot16<true>(q2, w0, w1, alpha);
+      } else {
+        part[j] = dot16<false>(q2, w0, 0u, alpha);
+      }
+    }
+  } else if constexpr (C::kQuant) {
+    // unfinished key group: exact bf16 keys from the residual
+#pragma unroll
+    for (int j = 0; j < TPL; ++j) {
+      const int t = r + TS * j;
+      float d = 0.f;
+      if (tok0 + t < nn) {
+        const uint4* kp = reinterpret_cast<const uint4*>(res + t * D + 16 * k);
+        const uint4 a = kp[0], c = kp[1];
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+        float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          s2 = __ffma2_rn(make_float2(qf[2 * i], qf[2 * i + 1]), make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
+        d = (s2.x + s2.y) * pow2i(-C::kE);
+      }
+      part[j] = d;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < TPL; ++j) {
+      const uint4* kp = reinterpret_cast<const uint4*>(st + ((TS * j) >> 4) * LOAD + R::kBfK +
+                                                       (r + ((TS * j) & 15)) * D * 2 + 32 * k);
+      const uint4 a = kp[0], c = kp[1];
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+      float2 s2 = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        s2 = __ffma2_rn(make_float2(qf[2 * i], qf[2 * i + 1]), make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
+      part[j] = s2.x + s2.y;
+    }
+  }
+  // all-reduce each token's logit over its CH lanes
+#pragma unroll
+  for (int j = 0; j < TPL; ++j)
+#pragma unroll
+    for (int o = 1; o < CH; o <<= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+
+  // ---- online softmax over the group (log2 units)
+  float gm = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < TPL; ++j)
+    if (!TAIL || tok0 + r + TS * j < nn) gm = fmaxf(gm, part[j]);
+#pragma unroll
+  for (int o = CH; o < 32; o <<= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+  gm *= esc;
+  if (gm > ws.m) {
+    const float c = fast_exp2(ws.m - gm);
+    ws.l *= c;
+    ws.beta *= c;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ws.acc[i] = __fmul2_rn(ws.acc[i], make_float2(c, c));
+    ws.m = gm;
+  }
+  // weights carry 2^kVSh (undone once at the end)
+  const float off = static_cast<float>(C::kVSh) - ws.m;
+  float wgt[TPL];
+#pragma unroll
+  for (int j = 0; j < TPL; ++j) {
+    wgt[j] = fast_exp2(fmaf(part[j], esc, off));
+    if (TAIL && tok0 + r + TS * j >= nn) wgt[j] = 0.f;
+    ws.l += wgt[j];
+  }
+  if constexpr (C::kLogits) {
+    float mine = part[0];
+#pragma unroll
+    for (int j = 1; j < TPL; ++j) mine = (j == k) ? part[j] : mine;
+    logits_g[r + TS * k] = mine * esc;
+  }
+
+  // ---- values
+#pragma unroll
+  for (int j = 0; j < TPL; ++j) {
+    if constexpr (C::kQuant) {
+      const uint8_t* row = rowbase + tok_off(j);
+      const uint32_t mv = *reinterpret_cast<const uint32_t*>(
+          st + ((TS * j) >> 4) * LOAD + R::kVMetaOff +
+          ((r + ((TS * j) & 15)) * (D / kGroup) + (k >> 1)) * 4);
+      float s = bf16_lo(mv), mn = bf16_hi(mv);
+      if (TAIL && tok0 + r + TS * j >= nn) s = mn = 0.f;
+      const uint32_t vh = *reinterpret_cast<const uint32_t*>(row + R::kVHi);
+      if constexpr (C::kFourV) {
+        const uint32_t vl = *reinterpret_cast<const uint32_t*>(row + R::kQ4VLo);
+        ws.beta = fmaf(wgt[j], mn, ws.beta);
+        axpy16<true>(ws.acc, wgt[j] * s, vh, vl);
+      } else if constexpr (C::kQ4) {
+        ws.beta = fmaf(wgt[j], fmaf(1.5f, s, mn), ws.beta);
+        axpy16<false>(ws.acc, wgt[j] * s, vh, 0u);
+      } else {
+        ws.beta = fmaf(wgt[j], mn, ws.beta);
+        axpy16<false>(ws.acc, wgt[j] * s, vh, 0u);
+      }
+    } else {
+      const uint4* vp = reinterpret_cast<const uint4*>(st + ((TS * j) >> 4) * LOAD + R::kBfV +
+                                                       (r + ((TS * j) & 15)) * D * 2 + 32 * k);
+      const uint4 a = vp[0], c = vp[1];
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+      const float2 ww = make_float2(wgt[j], wgt[j]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ws.acc[i] = __ffma2_rn(ww, make_float2(bf16_lo(w[i]), bf16_hi(w[i])), ws.acc[i]);
+    }
+  }
+}
+
+template <int KIND, int D, bool FULLV, bool CLUSTER>
+__global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams p) {
+  using C = Cfg<KIND, D, FULLV>;
+  using R = typename C::R;
+  constexpr int CH = C::kCH, TS = C::kTS, NSW = C::kNSW;
   constexpr int LOAD = C::kLoad, STAGE = C::kStage;
 
   extern __shared__ __align__(128) uint8_t smem[];
-  const Smem sp = smem_plan(STAGE, NS, p.chunk_groups, D, C::kLogits);
-  uint8_t* stages = smem + sp.stages;
-  const uint32_t full_bar = smem_addr(smem + sp.bars);
-  const uint32_t empty_bar = full_bar + 8 * NS;
-  int32_t* ids = reinterpret_cast<int32_t*>(smem + sp.ids);
+  const Smem sp = smem_plan(STAGE, NSW, p.chunk_groups, D, C::kLogits);
   float* logits = reinterpret_cast<float*>(smem + sp.logits);
   float* wscr = reinterpret_cast<float*>(smem + sp.wscr);
   float* cta_acc = reinterpret_cast<float*>(smem + sp.cta);
@@ -168,7 +322,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_allow_dependents();
 
-  // ---- this split's chunk of 32-token groups
+  // ---- this split's chunk of 32-token groups (seq_lens and the block table
+  //      are not written by the previous kernel: read before its completion)
   const int n = p.seq_lens[b];
   int bad = 0;
   if (n < 0 || n > p.max_seq_len || n > p.max_blocks * kBlock) bad = LOOPKV_DEVERR_SEQ_LEN;
@@ -180,262 +335,147 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   if (cg > p.chunk_groups) bad = LOOPKV_DEVERR_SEQ_LEN;
   const int n_blocks = (nn + kBlock - 1) / kBlock;
 
+  // this warp's ring and barriers
+  uint8_t* ring = smem + sp.rings + static_cast<size_t>(warp) * NSW * STAGE;
+  const uint32_t bar0 = smem_addr(smem + sp.bars) + 8 * NSW * warp;
+  if (lane == 0)
+    for (int i = 0; i < NSW; ++i) mbar_init(bar0 + 8 * i, 1);
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(full_bar + 8 * i, 1);
-      mbar_init(empty_bar + 8 * i, 1);
-    }
     cta_f[kSlotM] = -INFINITY;
     cta_f[kSlotL] = 0.f;
     cta_i[kSlotCount] = 0;
     cta_i[kSlotBad] = bad;
-    fence_mbar_init();
   }
+  fence_mbar_init();
   __syncthreads();
-  if (warp == kNW && !bad) {
-    for (int i = lane; i < 2 * cg; i += 32) {
-      const int lb = 2 * g0 + i;
-      int id = -1;
+
+  const int k = lane % CH, r = lane / CH;
+  WarpState ws;
+  ws.m = -INFINITY;
+  ws.l = 0.f;
+  ws.beta = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ws.acc[i] = make_float2(0.f, 0.f);
+
+  // groups of this warp: gi = warp + kNW * it
+  const int nit = (!bad && cg > warp) ? (cg - warp + kNW - 1) / kNW : 0;
+  const int g_unsafe = (nn - 1) / kGroup;  // may be written by the previous kernel
+  const uint64_t pol = l2_evict_first_policy();
+  const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+  // block ids of 16 iterations, two per iteration, spread over the lanes
+  auto load_ids = [&](int it0) {
+    const int it = it0 + (lane >> 1);
+    int id = -1;
+    if (it < nit) {
+      const int lb = 2 * (g0 + warp + kNW * it) + (lane & 1);
       if (lb < n_blocks) {
-        id = p.block_table[static_cast<size_t>(b) * p.max_blocks + lb];
-        if (id < 0 || id >= p.num_blocks) atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_BLOCK_ID);
+        id = table[lb];
+        if (id < 0 || id >= p.num_blocks) {
+          atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_BLOCK_ID);
+          id = -1;
+        }
       }
-      ids[i] = id;
     }
-  }
-  __syncthreads();
-  bad = cta_i[kSlotBad];
+    return id;
+  };
+  int ids = load_ids(0), ids_base = 0;
+  // issue the bulk copies of iteration `it` into its stage (all lanes call)
+  auto issue = [&](int it) {
+    if (it >= nit) return;
+    if (it - ids_base >= 16) {
+      ids_base += 16;
+      ids = load_ids(ids_base);
+    }
+    const int id0 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base));
+    const int id1 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base) + 1);
+    if (lane == 0) {
+      const int stage = it % NSW;
+      const uint32_t bar = bar0 + 8 * stage;
+      const uint32_t dst = smem_addr(ring + stage * STAGE);
+      const uint32_t bytes = (id0 >= 0 ? LOAD : 0) + (id1 >= 0 ? LOAD : 0);
+      mbar_arrive_expect_tx(bar, bytes);
+      if (id0 >= 0)
+        bulk_load(dst, p.arena + (static_cast<size_t>(id0) * p.H + h) * R::kBytes, LOAD, bar, pol);
+      if (id1 >= 0)
+        bulk_load(dst + LOAD, p.arena + (static_cast<size_t>(id1) * p.H + h) * R::kBytes, LOAD, bar, pol);
+    }
+  };
 
   // ---- pass 1
-  const int k = lane % CH, r = lane / CH;
-  float m_w = -INFINITY, l_w = 0.f, beta = 0.f;
-  float2 acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = make_float2(0.f, 0.f);
+  if (nit > 0) {
+    int issued = 0;
+    while (issued < NSW && issued < nit && g0 + warp + kNW * issued < g_unsafe) issue(issued++);
+    pdl_wait_prior_grid();  // q, the residual and the newest group may come from the previous kernel
+    while (issued < NSW) issue(issued++);
 
-  if (!bad && cg > 0) {
-    if (warp == kNW) {
-      if (lane == 0) {
-        // producer: blocks of groups before the one holding the newest token
-        // cannot be written by the previous kernel, so they stream at once.
-        const uint64_t pol = l2_evict_first_policy();
-        const int g_unsafe = (nn - 1) / kGroup;
-        bool waited = false;
-        for (int gi = 0; gi < cg; ++gi) {
-          const int stage = gi % NS;
-          if (gi >= NS && !mbar_wait(empty_bar + 8 * stage, ((gi / NS) - 1) & 1)) {
-            atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_TIMEOUT);
-            break;
-          }
-          const int G = g0 + gi;
-          if (!waited && G >= g_unsafe) {
-            pdl_wait_prior_grid();
-            waited = true;
-          }
-          const int nb = min(2, n_blocks - 2 * G);
-          mbar_arrive_expect_tx(full_bar + 8 * stage, nb * LOAD);
-          for (int blk = 0; blk < nb; ++blk)
-            bulk_load(smem_addr(stages + stage * STAGE + blk * LOAD),
-                      p.arena + (static_cast<size_t>(ids[2 * gi + blk]) * p.H + h) * R::kBytes,
-                      LOAD, full_bar + 8 * stage, pol);
-        }
+    // this lane's 16 query channels, in log2 units
+    float qf[16], qs[16];
+    {
+      const uint4* qp = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.H + h) * D + 16 * k);
+      const uint4 a = qp[0], c = qp[1];
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        qf[2 * i] = bf16_lo(w[i]) * p.sm_scale_log2;
+        qf[2 * i + 1] = bf16_hi(w[i]) * p.sm_scale_log2;
       }
-    } else {
-      pdl_wait_prior_grid();  // q and the key residual may come from the previous kernel
-      // this lane's 16 query channels, in log2 units
-      float qf[16], qs[16];
-      {
-        const uint4* qp = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.H + h) * D + 16 * k);
-        const uint4 a = qp[0], c = qp[1];
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          qf[2 * i] = bf16_lo(w[i]) * p.sm_scale_log2;
-          qf[2 * i + 1] = bf16_hi(w[i]) * p.sm_scale_log2;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          qs[i] = qf[i] * pow2i(149 - (C::kQ4 ? pos4(i) : pos2(i)) - C::kE);
+      for (int i = 0; i < 16; ++i) qs[i] = qf[i] * pow2i(149 - (C::kQ4 ? pos4(i) : pos2(i)) - C::kE);
+    }
+    const __nv_bfloat16* res = C::kQuant ? p.residual + (static_cast<size_t>(b) * p.H + h) * kGroup * D : nullptr;
+
+    for (int it = 0; it < nit; ++it) {
+      const int stage = it % NSW;
+      if (!mbar_wait(bar0 + 8 * stage, (it / NSW) & 1)) {
+        atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_TIMEOUT);
+        break;
       }
-      const float esc = pow2i(C::kE), inv_esc = pow2i(-C::kE);
-
-      for (int gi = warp; gi < cg; gi += kNW) {
-        const int stage = gi % NS;
-        if (!mbar_wait(full_bar + 8 * stage, (gi / NS) & 1)) {
-          atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_TIMEOUT);
-          break;
-        }
-        const uint8_t* st = stages + stage * STAGE;
-        const int tok0 = (g0 + gi) * kGroup;
-        const bool tail = tok0 + kGroup > nn;
-
-        // ---- keys -> logits (scaled by 2^-E)
-        float part[TPL];
-        if constexpr (C::kQuant) {
-          if (!tail) {
-            const uint8_t* km = st + ((16 * k < D / 2) ? 0 : LOAD) + R::kKMetaOff + ((16 * k) % (D / 2)) * 4;
-            float q2[16];
-            float alpha = 0.f;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const uint4 mw = reinterpret_cast<const uint4*>(km)[v];
-              const uint32_t ws[4] = {mw.x, mw.y, mw.z, mw.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int i = 4 * v + u;
-                q2[i] = qs[i] * bf16_lo(ws[u]);
-                alpha = fmaf(qf[i], bf16_hi(ws[u]), alpha);
-              }
-            }
-            alpha *= inv_esc;
-#pragma unroll
-            for (int j = 0; j < TPL; ++j) {
-              const int t = r + TS * j;
-              const uint8_t* row = st + (t >> 4) * LOAD + (t & 15) * R::kRow + 4 * k;
-              const uint32_t w0 = *reinterpret_cast<const uint32_t*>(row + R::kKHi);
-              if constexpr (C::kQ4) {
-                const uint32_t w1 = *reinterpret_cast<const uint32_t*>(row + R::kQ4KLo);
-                part[j] = dot16<true>(q2, w0, w1, alpha);
-              } else {
-                part[j] = dot16<false>(q2, w0, 0u, alpha);
-              }
-            }
-          } else {
-            // unfinished key group: exact bf16 keys from the residual
-            const __nv_bfloat16* res = p.residual + (static_cast<size_t>(b) * p.H + h) * kGroup * D + 16 * k;
-#pragma unroll
-            for (int j = 0; j < TPL; ++j) {
-              const int t = r + TS * j;
-              float d = 0.f;
-              if (tok0 + t < nn) {
-                const uint4* kp = reinterpret_cast<const uint4*>(res + t * D);
-                const uint4 a = kp[0], c = kp[1];
-                const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-                float2 s2 = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                  s2 = __ffma2_rn(make_float2(qf[2 * i], qf[2 * i + 1]), make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
-                d = (s2.x + s2.y) * inv_esc;
-              }
-              part[j] = d;
-            }
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < TPL; ++j) {
-            const int t = r + TS * j;
-            const uint4* kp = reinterpret_cast<const uint4*>(st + (t >> 4) * LOAD + R::kBfK + (t & 15) * D * 2 + 32 * k);
-            const uint4 a = kp[0], c = kp[1];
-            const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-            float2 s2 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              s2 = __ffma2_rn(make_float2(qf[2 * i], qf[2 * i + 1]), make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
-            part[j] = s2.x + s2.y;
-          }
-        }
-        // all-reduce each token's logit over its CH lanes
-#pragma unroll
-        for (int j = 0; j < TPL; ++j)
-#pragma unroll
-          for (int o = 1; o < CH; o <<= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
-
-        // ---- online softmax over the group (log2 units)
-        float gm = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < TPL; ++j)
-          if (tok0 + r + TS * j < nn) gm = fmaxf(gm, part[j]);
-#pragma unroll
-        for (int o = CH; o < 32; o <<= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
-        gm *= esc;
-        if (gm > m_w) {
-          const float c = fast_exp2(m_w - gm);
-          l_w *= c;
-          beta *= c;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = make_float2(acc[i].x * c, acc[i].y * c);
-          m_w = gm;
-        }
-        float wgt[TPL];
-#pragma unroll
-        for (int j = 0; j < TPL; ++j) {
-          wgt[j] = (tok0 + r + TS * j < nn) ? fast_exp2(fmaf(part[j], esc, -m_w)) : 0.f;
-          l_w += wgt[j];
-        }
-        if constexpr (C::kLogits) {
-          float mine = part[0];
-#pragma unroll
-          for (int j = 1; j < TPL; ++j) mine = (j == k) ? part[j] : mine;
-          logits[gi * kGroup + r + TS * k] = mine * esc;
-        }
-
-        // ---- values
-#pragma unroll
-        for (int j = 0; j < TPL; ++j) {
-          const int t = r + TS * j;
-          if constexpr (C::kQuant) {
-            const uint8_t* blk = st + (t >> 4) * LOAD;
-            const uint32_t mv = *reinterpret_cast<const uint32_t*>(blk + R::kVMetaOff + ((t & 15) * (D / kGroup) + (k >> 1)) * 4);
-            const bool ok = !tail || (tok0 + t < nn);
-            const float s = ok ? bf16_lo(mv) : 0.f;
-            const float mn = ok ? bf16_hi(mv) : 0.f;
-            const uint8_t* row = blk + (t & 15) * R::kRow + 4 * k;
-            const uint32_t vh = *reinterpret_cast<const uint32_t*>(row + R::kVHi);
-            if constexpr (C::kQ4 && FULLV) {
-              const uint32_t vl = *reinterpret_cast<const uint32_t*>(row + R::kQ4VLo);
-              beta = fmaf(wgt[j], mn, beta);
-              axpy16<true>(acc, wgt[j] * s * pow2i(85), vh, vl);
-            } else if constexpr (C::kQ4) {
-              beta = fmaf(wgt[j], fmaf(1.5f, s, mn), beta);
-              axpy16<false>(acc, wgt[j] * s * pow2i(87), vh, 0u);
-            } else {
-              beta = fmaf(wgt[j], mn, beta);
-              axpy16<false>(acc, wgt[j] * s * pow2i(85), vh, 0u);
-            }
-          } else {
-            const uint4* vp = reinterpret_cast<const uint4*>(st + (t >> 4) * LOAD + R::kBfV + (t & 15) * D * 2 + 32 * k);
-            const uint4 a = vp[0], c = vp[1];
-            const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-            const float2 ww = make_float2(wgt[j], wgt[j]);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = __ffma2_rn(ww, make_float2(bf16_lo(w[i]), bf16_hi(w[i])), acc[i]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty_bar + 8 * stage);
-      }
+      const int gi = warp + kNW * it;
+      const int tok0 = (g0 + gi) * kGroup;
+      const uint8_t* st = ring + stage * STAGE;
+      float* lg = logits + gi * kGroup;
+      if (tok0 + kGroup <= nn)
+        group_step<KIND, D, FULLV, false>(st, qf, qs, res, tok0, nn, r, k, lg, ws);
+      else
+        group_step<KIND, D, FULLV, true>(st, qf, qs, res, tok0, nn, r, k, lg, ws);
+      __syncwarp();
+      if (lane == 0) fence_proxy_async_smem();
+      issue(it + NSW);
     }
   }
+  pdl_wait_prior_grid();  // nothing below may run ahead of the previous kernel
 
   // ---- warp results: true per-channel sums, reduced over token sub-groups
-  if (warp < kNW) {
+  {
+    const float unsh = pow2i(-C::kVSh);
     float o[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if constexpr (C::kQuant) {
-        const int pa = (C::kQ4 && FULLV) ? pos4(2 * i) : pos2(2 * i);
-        const int pb = (C::kQ4 && FULLV) ? pos4(2 * i + 1) : pos2(2 * i + 1);
-        o[2 * i] = fmaf(acc[i].x, pow2i(64 - pa), beta);
-        o[2 * i + 1] = fmaf(acc[i].y, pow2i(64 - pb), beta);
+        const int pa = C::kFourV ? pos4(2 * i) : pos2(2 * i);
+        const int pb = C::kFourV ? pos4(2 * i + 1) : pos2(2 * i + 1);
+        o[2 * i] = fmaf(ws.acc[i].x, pow2i(64 - pa), ws.beta * unsh);
+        o[2 * i + 1] = fmaf(ws.acc[i].y, pow2i(64 - pb), ws.beta * unsh);
       } else {
-        o[2 * i] = acc[i].x;
-        o[2 * i + 1] = acc[i].y;
+        o[2 * i] = ws.acc[i].x;
+        o[2 * i + 1] = ws.acc[i].y;
       }
     }
+    float l = ws.l * unsh;
 #pragma unroll
     for (int off = CH; off < 32; off <<= 1) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) o[i] += __shfl_xor_sync(0xffffffffu, o[i], off);
-      l_w += __shfl_xor_sync(0xffffffffu, l_w, off);
+      l += __shfl_xor_sync(0xffffffffu, l, off);
     }
-    float* ws = wscr + warp * (D + 4);
+    float* wsc = wscr + warp * (D + 4);
     if (r == 0) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) ws[16 * k + i] = o[i];
+      for (int i = 0; i < 16; ++i) wsc[16 * k + i] = o[i];
     }
     if (lane == 0) {
-      ws[D] = m_w;
-      ws[D + 1] = l_w;
+      wsc[D] = ws.m;
+      wsc[D + 1] = l;
     }
   }
   __syncthreads();
@@ -497,9 +537,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   const float inv_z = live ? 1.f / z : 0.f;
 
   // ---- pass 2: low-plane selection and gather (4-bit sources)
-  pdl_wait_prior_grid();  // nothing below writes memory the previous kernel may still use
   const bool want_mask = p.sel_mask != nullptr || p.sel_count != nullptr;
-  if (warp < kNW && live && ((C::kLogits && p.tau < INFINITY) || want_mask)) {
+  if (live && ((C::kLogits && p.tau < INFINITY) || want_mask)) {
     const float m_c = cta_f[kSlotM];
     float corr[16];
 #pragma unroll
@@ -528,14 +567,14 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
           const int t = (my < nsel) ? (__ffs(mm) - 1) : 0;
           const float lt = __shfl_sync(0xffffffffu, lg, t);
           if (my < nsel) {
-            const int phys = ids[2 * gi + (t >> 4)];
+            const int phys = p.block_table[static_cast<size_t>(b) * p.max_blocks + 2 * (g0 + gi) + (t >> 4)];
             const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
             const uint32_t lo = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VLo + (t & 15) * R::kRow + 4 * k);
             const uint32_t mv = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VMeta + ((t & 15) * (D / kGroup) + (k >> 1)) * 4);
-            const float ws = fast_exp2(lt - m_c) * bf16_lo(mv);
+            const float wsel = fast_exp2(lt - m_c) * bf16_lo(mv);
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              corr[i] = fmaf(ws, static_cast<float>((lo >> (2 * i)) & 3u) - 1.5f, corr[i]);
+              corr[i] = fmaf(wsel, static_cast<float>((lo >> (2 * i)) & 3u) - 1.5f, corr[i]);
           }
         }
       }
@@ -563,8 +602,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       for (int s = 0; s < S; ++s) {
         float ms, as;
         if constexpr (CLUSTER) {
-          const uint32_t pa = peer_addr(my_f, s);
-          ms = ld_peer_f32(pa + 4 * kSlotM);
+          ms = ld_peer_f32(peer_addr(my_f, s) + 4 * kSlotM);
           as = ld_peer_f32(peer_addr(smem_addr(cta_acc + c), s));
         } else {
           ms = cta_f[kSlotM];
@@ -579,7 +617,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   if (split == 0 && threadIdx.x == 0) {
     if (p.sel_count) {
       int total = 0;
-      if (live && (C::kQ4)) {
+      if (live && C::kQ4) {
         for (int s = 0; s < S; ++s) {
           if constexpr (CLUSTER) total += ld_peer_s32(peer_addr(smem_addr(&cta_i[kSlotCount]), s));
           else total += cta_i[kSlotCount];
@@ -593,17 +631,34 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 }
 
 template <int KIND, int D, bool FULLV, bool CLUSTER>
-cudaError_t launch_t(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
+size_t smem_bytes_t(int cg) {
   using C = Cfg<KIND, D, FULLV>;
-  const Smem sp = smem_plan(C::kStage, C::kNS, p.chunk_groups, D, C::kLogits);
-  if (sp.total > 227u * 1024u) return cudaErrorInvalidValue;
+  return smem_plan(C::kStage, C::kNSW, cg, D, C::kLogits).total;
+}
+
+template <int KIND, int D, bool FULLV, bool CLUSTER>
+int occupancy_t(int cg) {
+  int blocks = 0;
+  const size_t smem = smem_bytes_t<KIND, D, FULLV, CLUSTER>(cg);
+  if (smem > 227u * 1024u) return 0;
   auto kern = decode_kernel<KIND, D, FULLV, CLUSTER>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sp.total));
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kThreads, smem) != cudaSuccess) return 0;
+  return blocks;
+}
+
+template <int KIND, int D, bool FULLV, bool CLUSTER>
+cudaError_t launch_t(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
+  const size_t smem = smem_bytes_t<KIND, D, FULLV, CLUSTER>(p.chunk_groups);
+  if (smem > 227u * 1024u) return cudaErrorInvalidValue;
+  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(splits, p.H, batch);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = sp.total;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   int na = 0;
@@ -630,23 +685,24 @@ cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t 
                     : launch_t<KIND, D, FULLV, false>(p, batch, splits, stream, pdl);
 }
 
-}  // namespace
-
-namespace {
-size_t smem_for(int kind, int head_dim, bool full_values, int cg) {
-  int rec, load, ns = 8;
-  const int plane = 16 * head_dim / 4, kmeta = head_dim * 2, vmeta = 16 * (head_dim / 32) * 4;
-  if (kind == LOOPKV_CELL_Q4) {
-    rec = 4 * plane + kmeta + vmeta;
-    load = full_values ? rec : rec - plane;
-  } else if (kind == LOOPKV_CELL_Q2) {
-    load = 2 * plane + kmeta + vmeta;
-  } else {
-    load = 64 * head_dim;
-    ns = 4;
-  }
-  return smem_plan(2 * load, ns, cg, head_dim, kind == LOOPKV_CELL_Q4 && !full_values).total;
+template <int KIND, int D, bool FULLV>
+int occupancy_c(bool cluster, int cg) {
+  return cluster ? occupancy_t<KIND, D, FULLV, true>(cg) : occupancy_t<KIND, D, FULLV, false>(cg);
 }
+
+// CTAs of one decode instantiation that fit on one SM.
+int blocks_per_sm(int kind, int d, bool cluster, int cg) {
+  switch (kind * 1000 + d) {
+    case LOOPKV_CELL_Q4 * 1000 + 128: return occupancy_c<LOOPKV_CELL_Q4, 128, false>(cluster, cg);
+    case LOOPKV_CELL_Q4 * 1000 + 64: return occupancy_c<LOOPKV_CELL_Q4, 64, false>(cluster, cg);
+    case LOOPKV_CELL_Q2 * 1000 + 128: return occupancy_c<LOOPKV_CELL_Q2, 128, false>(cluster, cg);
+    case LOOPKV_CELL_Q2 * 1000 + 64: return occupancy_c<LOOPKV_CELL_Q2, 64, false>(cluster, cg);
+    case LOOPKV_CELL_BF16 * 1000 + 128: return occupancy_c<LOOPKV_CELL_BF16, 128, false>(cluster, cg);
+    case LOOPKV_CELL_BF16 * 1000 + 64: return occupancy_c<LOOPKV_CELL_BF16, 64, false>(cluster, cg);
+    default: return 0;
+  }
+}
+
 }  // namespace
 
 // Largest context one split may hold (its logits live in shared memory).
@@ -663,11 +719,11 @@ int decode_splits(int kind, int head_dim, int batch, int heads, int max_seq_len)
   int best = min_s;
   double best_eff = -1.0;
   for (int s = min_s; s <= 8; s <<= 1) {
-    if (s > min_s && groups < 4 * s) break;  // keep at least 4 groups per split
+    if (s > min_s && groups < 2 * kNW * s) break;  // keep >= 2 groups per warp
     const int cg = (groups + s - 1) / s;
-    const size_t smem = smem_for(kind, head_dim, false, cg) + 1024;
-    const long per_sm = std::min<long>(4, static_cast<long>((228u * 1024u) / smem));
-    const long slots = static_cast<long>(sms) * std::max<long>(1, per_sm);
+    int per_sm = blocks_per_sm(kind, head_dim, s > 1, cg);
+    if (per_sm <= 0) per_sm = 4;  // no device: a fixed guess keeps the choice deterministic
+    const long slots = static_cast<long>(sms) * per_sm;
     const long ctas = pairs * s;
     const long waves = (ctas + slots - 1) / slots;
     const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);

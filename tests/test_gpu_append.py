@@ -20,26 +20,29 @@ def _small(d, lens, paging="shuffled", seed=5, heads=3):
 
 def _ragged_append(kv, k, v, lens, table_d, rounds):
     """Append so that sequence b ends with lens[b] tokens, in several calls
-    whose start positions differ per sequence (negative = skipped)."""
+    whose start positions differ per sequence (negative = skipped): at every
+    cut, sequences that still lack tokens take a common chunk T."""
     from mixed_precision_kv_loopkv_b200 import loopkv_quantize_append
     B = k.shape[0]
     have = [0] * B
     for cut in rounds:
-        T = max(min(cut, lens[b]) - have[b] for b in range(B))
-        if T <= 0:
-            continue
-        starts, kr, vr = [], torch.zeros_like(k[:, :T]), torch.zeros_like(v[:, :T])
-        for b in range(B):
-            take = min(cut, lens[b]) - have[b]
-            if take == T:
-                starts.append(have[b])
-                kr[b] = k[b, have[b]: have[b] + T]
-                vr[b] = v[b, have[b]: have[b] + T]
-                have[b] += T
-            else:
-                starts.append(-1)
-        st = torch.tensor(starts, dtype=torch.int32, device=k.device)
-        loopkv_quantize_append(kv, 0, 0, kr.contiguous(), vr.contiguous(), table_d, st)
+        while True:
+            takes = [min(cut, lens[b]) - have[b] for b in range(B)]
+            pos = [t for t in takes if t > 0]
+            if not pos:
+                break
+            T = min(pos)
+            starts, kr, vr = [], torch.zeros_like(k[:, :T]), torch.zeros_like(v[:, :T])
+            for b in range(B):
+                if takes[b] > 0:
+                    starts.append(have[b])
+                    kr[b] = k[b, have[b]: have[b] + T]
+                    vr[b] = v[b, have[b]: have[b] + T]
+                    have[b] += T
+                else:
+                    starts.append(-1)
+            st = torch.tensor(starts, dtype=torch.int32, device=k.device)
+            loopkv_quantize_append(kv, 0, 0, kr.contiguous(), vr.contiguous(), table_d, st)
     return have
 
 
