@@ -197,8 +197,7 @@ def profiled_traffic(workload: str):
 # ----------------------------------------------------------------- workload setup
 
 def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0):
-    from mixed_precision_kv_loopkv_b200 import (LOOPKV_FLAG_PDL, KVCells, LoopedDecodeStep,
-                                                loopkv_quantize_append)
+    from mixed_precision_kv_loopkv_b200 import LOOPKV_FLAG_PDL, KVCells, LoopedDecodeStep, prefill
     from workload import block_table_for, cell_kv, cell_new_token, cell_query, make_plan, seq_lens_for
 
     plan = make_plan(w)
@@ -213,13 +212,15 @@ def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0):
                  table_np.shape[1], flags=LOOPKV_FLAG_PDL if pdl else 0, decode_splits=splits,
                  allocate=set(run))
     table = torch.from_numpy(table_np).cuda()
-    zero = torch.zeros(w.batch, dtype=torch.int32, device="cuda")
     stored = [c for c in run if plan[c] != "reuse"]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
     for c in stored:
         loop, layer = divmod(c, w.num_layers)
         k, v = cell_kv(w, loop, layer, device="cuda")
-        loopkv_quantize_append(kv, loop, layer, k, v, table, zero)
+        prefill(kv, loop, layer, k, v, table, lens, err_flag=err)
         del k, v
+    if int(err):
+        raise RuntimeError(f"prefill flagged device error {int(err)}")
     q_all = torch.stack([cell_query(w, *divmod(c, w.num_layers), device="cuda") for c in range(C)])
     kn_all = torch.empty((len(stored), w.batch, 1, w.num_heads, w.head_dim), dtype=torch.bfloat16,
                          device="cuda")

@@ -29,4 +29,4 @@ from .loopkv import (  # noqa: F401
     loopkv_status_string,
     mask_words,
 )
-from .step import LoopedDecodeStep  # noqa: F401
+from .step import LoopedDecodeStep, prefill  # noqa: F401

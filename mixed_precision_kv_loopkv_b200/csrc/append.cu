@@ -78,9 +78,11 @@ __device__ __forceinline__ uint8_t* record_of(const AppendParams& p, int b, int 
 template <int KIND, int D>
 __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
   using R = Rec<KIND, D>;
-  // The new tokens may be produced by the kernel right before this one.
-  pdl_wait_prior_grid();
+  // Let the next kernel (a decode of this cell) launch and stream the cache
+  // blocks this kernel does not write; then wait for the kernel before this
+  // one, which may produce the new tokens.
   pdl_allow_dependents();
+  pdl_wait_prior_grid();
 
   const int h = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

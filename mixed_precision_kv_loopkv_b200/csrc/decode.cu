@@ -70,30 +70,34 @@ __device__ __forceinline__ void combine_planes(uint32_t hi, uint32_t lo, uint32_
   odd = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
 }
 
-// Dot product of 16 subnormal code views with 16 pre-scaled coefficients
-// (pairs of channels 2p, 2p+1).
+// Dot product of the subnormal code views of one 16-channel word with 8
+// coefficient pairs (channels 2p, 2p+1), two short chains.
 template <bool FOUR>
-__device__ __forceinline__ float dot16(const float2* c, uint32_t a, uint32_t b, float init) {
-  float2 acc = make_float2(init, 0.f);
+__device__ __forceinline__ float2 dot16(const float2* c, uint32_t a, uint32_t b, float2 acc0) {
+  float2 acc1 = make_float2(0.f, 0.f);
   if constexpr (FOUR) {  // a, b = high / low plane words
     uint32_t e, o;
     combine_planes(a, b, e, o);
     const uint32_t e20 = e >> 20, o20 = o >> 20;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) acc = __ffma2_rn(c[m], make_float2(nib(e, e20, m), nib(o, o20, m)), acc);
+    for (int m = 0; m < 8; m += 2) {
+      acc0 = __ffma2_rn(c[m], make_float2(nib(e, e20, m), nib(o, o20, m)), acc0);
+      acc1 = __ffma2_rn(c[m + 1], make_float2(nib(e, e20, m + 1), nib(o, o20, m + 1)), acc1);
+    }
   } else {  // a = 2-bit plane word
     const uint32_t a22 = a >> 22;
 #pragma unroll
-    for (int p = 0; p < 8; ++p)
-      acc = __ffma2_rn(c[p], make_float2(fld2(a, a22, 2 * p), fld2(a, a22, 2 * p + 1)), acc);
+    for (int p = 0; p < 8; p += 2) {
+      acc0 = __ffma2_rn(c[p], make_float2(fld2(a, a22, 2 * p), fld2(a, a22, 2 * p + 1)), acc0);
+      acc1 = __ffma2_rn(c[p + 1], make_float2(fld2(a, a22, 2 * p + 2), fld2(a, a22, 2 * p + 3)), acc1);
+    }
   }
-  return acc.x + acc.y;
+  return __fadd2_rn(acc0, acc1);
 }
 
-// acc[p] += w * (codes of channels 2p, 2p+1)
+// acc[p] += w * (codes of channels 2p, 2p+1) of one 16-channel word
 template <bool FOUR>
-__device__ __forceinline__ void axpy16(float2* acc, float w, uint32_t a, uint32_t b) {
-  const float2 ww = make_float2(w, w);
+__device__ __forceinline__ void axpy16(float2* acc, float2 ww, uint32_t a, uint32_t b) {
   if constexpr (FOUR) {
     uint32_t e, o;
     combine_planes(a, b, e, o);
@@ -115,11 +119,16 @@ struct Cfg {
   static constexpr bool kQ4 = KIND == LOOPKV_CELL_Q4;
   // bytes of one block record streamed in pass 1
   static constexpr int kLoad = kQ4 ? (FULLV ? R::kBytes : R::kQ4VLo) : R::kBytes;
-  static constexpr int kStage = 2 * kLoad;                 // one 32-token group
+  // one 32-token group: two block prefixes, the second shifted by 64 B so the
+  // same offsets of the two halves fall in different shared-memory banks
+  static constexpr int kHalf = kLoad + 64;
+  static constexpr int kStage = kHalf + kLoad;
   static constexpr int kNSW = kQuant ? 3 : 2;              // ring stages per warp
-  static constexpr int kCH = D / 16;                       // lanes per token
+  static constexpr int kCH = 4;                            // lanes per token
+  static constexpr int kCW = D / kCH;                      // channels per lane
+  static constexpr int kNWRD = kCW / 16;                   // plane words per lane and token
   static constexpr int kTS = 32 / kCH;                     // token sub-groups per warp
-  static constexpr int kTPL = kCH;                         // tokens per lane per group
+  static constexpr int kTPL = 32 / kTS;                    // tokens per lane per group
   static constexpr int kE = kQuant ? kExpOff : 0;
   // power of two folded into the softmax weight for the value products
   static constexpr int kVSh = !kQuant ? 0 : (kQ4 && !FULLV) ? 87 : 85;
@@ -128,17 +137,22 @@ struct Cfg {
 };
 
 // Shared-memory carve-up (bytes), identical on host and device.
+// After pass 1 a warp's ring is idle: its result scratch (wscr) lives at the
+// start of its own ring, and the CTA accumulators (used after a CTA barrier)
+// in warp 1's ring past that warp's scratch.
 struct Smem {
-  size_t rings, bars, logits, wscr, cta, total;
+  size_t rings, ring_bytes, bars, qconst, q2buf, logits, scal, total;
 };
 __host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int d, bool logits) {
   Smem s;
   s.rings = 0;
-  s.bars = s.rings + static_cast<size_t>(stage_bytes) * nsw * kNW;
-  s.logits = s.bars + 8 * nsw * kNW;
-  s.wscr = s.logits + (logits ? 128 * static_cast<size_t>(cg) : 0);
-  s.cta = s.wscr + static_cast<size_t>(kNW) * (d + 4) * 4;
-  s.total = s.cta + static_cast<size_t>(d + 4) * 4;
+  s.ring_bytes = static_cast<size_t>(stage_bytes) * nsw;
+  s.bars = s.rings + s.ring_bytes * kNW;
+  s.qconst = s.bars + 8 * nsw * kNW;                       // qf[D], qs[D]
+  s.q2buf = s.qconst + static_cast<size_t>(8) * d;         // per warp: 128 floats, swizzled
+  s.logits = s.q2buf + static_cast<size_t>(4) * 128 * kNW;
+  s.scal = s.logits + (logits ? 128 * static_cast<size_t>(cg) : 0);  // CTA scalars
+  s.total = s.scal + 16;
   return s;
 }
 
@@ -146,72 +160,114 @@ __host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int 
 enum { kSlotM = 0, kSlotL = 1, kSlotCount = 2, kSlotBad = 3 };
 
 // Per-lane running state of one warp's online softmax.
+template <int CW>
 struct WarpState {
   float m, l, beta;
-  float2 acc[8];
+  float2 acc[CW / 2];
 };
 
-// One 32-token group.  Lane (r, k): channels 16k..16k+15 of tokens
-// r + TS*j (j < TPL).  TAIL: the sequence's unfinished key group, keys from
-// the exact residual and tokens past the end masked.
+// Slot (in floats) of the 16-byte piece v (channels CW*k + 4v .. +3) in a
+// warp's q2 buffer: per-chunk reads (fixed v, k = 0..3) hit distinct bank
+// groups; the cooperative writes conflict at most two ways.
+template <int CW>
+__device__ __forceinline__ int q2_slot(int k, int v) { return v * 16 + ((k + v) & 3) * 4; }
+
+// One 32-token group.  Lane (r, k), r = lane / 4, k = lane % 4: channels
+// CW*k .. CW*k + CW - 1 of tokens r + 8j (j < 4).  TAIL: the sequence's
+// unfinished key group: keys from the exact residual, tokens past the end
+// masked.
 template <int KIND, int D, bool FULLV, bool TAIL>
-__device__ __forceinline__ void group_step(const uint8_t* st, const float* qf, const float* qs,
-                                           const __nv_bfloat16* res, int tok0, int nn, int r, int k,
-                                           float* logits_g, WarpState& ws) {
+__device__ __forceinline__ void group_step(const uint8_t* st, const float* qconst, float* q2buf,
+                                           const float* qfr, const __nv_bfloat16* res, int tok0, int nn,
+                                           int lane, int r, int k, float* logits_g,
+                                           WarpState<Cfg<KIND, D, FULLV>::kCW>& ws) {
   using C = Cfg<KIND, D, FULLV>;
   using R = typename C::R;
-  constexpr int CH = C::kCH, TS = C::kTS, TPL = C::kTPL, LOAD = C::kLoad;
+  constexpr int CH = C::kCH, CW = C::kCW, NWRD = C::kNWRD, TS = C::kTS, TPL = C::kTPL, HALF = C::kHalf;
   const float esc = pow2i(C::kE);
 
-  // this lane's row word of token j: rowbase + offset(j), a compile-time offset
-  const uint8_t* rowbase = st + r * R::kRow + 4 * k;
-  auto tok_off = [](int j) { return ((TS * j) >> 4) * LOAD + ((TS * j) & 15) * R::kRow; };
+  // this lane's plane words of token j: rowbase + a compile-time offset
+  const uint8_t* rowbase = st + r * R::kRow + 4 * NWRD * k;
+  auto tok_off = [](int j) { return ((TS * j) >> 4) * HALF + ((TS * j) & 15) * R::kRow; };
+  auto plane_words = [&](int j, int section, uint32_t* w) {
+    const uint8_t* a = rowbase + tok_off(j) + section;
+    if constexpr (NWRD == 2) {
+      const uint2 x = *reinterpret_cast<const uint2*>(a);
+      w[0] = x.x;
+      w[1] = x.y;
+    } else {
+      w[0] = *reinterpret_cast<const uint32_t*>(a);
+    }
+  };
 
   // ---- keys -> logits (scaled by 2^-E)
   float part[TPL];
   if constexpr (C::kQuant && !TAIL) {
-    const uint8_t* km = st + ((16 * k < D / 2) ? 0 : LOAD) + R::kKMetaOff + ((16 * k) % (D / 2)) * 4;
-    float2 q2[8];
-    float2 al = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint4 mw = reinterpret_cast<const uint4*>(km)[v];
-      const uint32_t w4[4] = {mw.x, mw.y, mw.z, mw.w};
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int i = 4 * v + 2 * u;
-        q2[i / 2] = __fmul2_rn(make_float2(qs[i], qs[i + 1]),
-                               make_float2(bf16_lo(w4[2 * u]), bf16_lo(w4[2 * u + 1])));
-        al = __ffma2_rn(make_float2(qf[i], qf[i + 1]),
-                        make_float2(bf16_hi(w4[2 * u]), bf16_hi(w4[2 * u + 1])), al);
+    // cooperative key coefficients of this group: lane l owns channels
+    // 4l..4l+3 (contiguous meta, conflict-free), q2 = qs * scale, and its
+    // share of alpha = sum_c qf_c * min_c
+    float alpha;
+    {
+      constexpr int kLanesUsed = D / 4;
+      float a4 = 0.f;
+      if (kLanesUsed == 32 || lane < kLanesUsed) {
+        const int c0 = 4 * lane;
+        const uint4 mw = *reinterpret_cast<const uint4*>(st + ((c0 < D / 2) ? 0 : HALF) + R::kKMetaOff +
+                                                         (c0 % (D / 2)) * 4);
+        const float4 qfv = *reinterpret_cast<const float4*>(qconst + c0);
+        const float4 qsv = *reinterpret_cast<const float4*>(qconst + D + c0);
+        const float2 q01 = __fmul2_rn(make_float2(qsv.x, qsv.y), make_float2(bf16_lo(mw.x), bf16_lo(mw.y)));
+        const float2 q23 = __fmul2_rn(make_float2(qsv.z, qsv.w), make_float2(bf16_lo(mw.z), bf16_lo(mw.w)));
+        float2 a2 = __fmul2_rn(make_float2(qfv.x, qfv.y), make_float2(bf16_hi(mw.x), bf16_hi(mw.y)));
+        a2 = __ffma2_rn(make_float2(qfv.z, qfv.w), make_float2(bf16_hi(mw.z), bf16_hi(mw.w)), a2);
+        a4 = a2.x + a2.y;
+        *reinterpret_cast<float4*>(q2buf + q2_slot<CW>(c0 / CW, (c0 % CW) / 4)) =
+            make_float4(q01.x, q01.y, q23.x, q23.y);
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a4 += __shfl_xor_sync(0xffffffffu, a4, o);
+      alpha = a4;
     }
-    const float alpha = (al.x + al.y) * pow2i(-C::kE);
+    __syncwarp();
+    float2 q2[CW / 2];
+#pragma unroll
+    for (int v = 0; v < CW / 4; ++v) {
+      const float4 x = *reinterpret_cast<const float4*>(q2buf + q2_slot<CW>(k, v));
+      q2[2 * v] = make_float2(x.x, x.y);
+      q2[2 * v + 1] = make_float2(x.z, x.w);
+    }
+    // each of the CH lanes of a token starts from alpha / CH (exact: CH is a
+    // power of two), so the all-reduce below adds alpha exactly once
+    alpha *= pow2i(-C::kE) / CH;
 #pragma unroll
     for (int j = 0; j < TPL; ++j) {
-      const uint8_t* row = rowbase + tok_off(j);
-      const uint32_t w0 = *reinterpret_cast<const uint32_t*>(row + R::kKHi);
-      if constexpr (C::kQ4) {
-        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(row + R::kQ4KLo);
-        part[j] = dot16<true>(q2, w0, w1, alpha);
-      } else {
-        part[j] = dot16<false>(q2, w0, 0u, alpha);
-      }
+      uint32_t hi[NWRD], lo[NWRD];
+      plane_words(j, R::kKHi, hi);
+      if constexpr (C::kQ4) plane_words(j, R::kQ4KLo, lo);
+      float2 d = make_float2(alpha, 0.f);
+#pragma unroll
+      for (int u = 0; u < NWRD; ++u) d = dot16<C::kQ4>(q2 + 8 * u, hi[u], C::kQ4 ? lo[u] : 0u, d);
+      part[j] = d.x + d.y;
     }
   } else if constexpr (C::kQuant) {
     // unfinished key group: exact bf16 keys from the residual
+    const float* qf = qconst + CW * k;
 #pragma unroll
     for (int j = 0; j < TPL; ++j) {
       const int t = r + TS * j;
       float d = 0.f;
       if (tok0 + t < nn) {
-        const uint4* kp = reinterpret_cast<const uint4*>(res + t * D + 16 * k);
-        const uint4 a = kp[0], c = kp[1];
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+        const uint4* kp = reinterpret_cast<const uint4*>(res + t * D + CW * k);
         float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          s2 = __ffma2_rn(make_float2(qf[2 * i], qf[2 * i + 1]), make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
+        for (int v = 0; v < CW / 8; ++v) {
+          const uint4 a = kp[v];
+          const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            s2 = __ffma2_rn(make_float2(qf[8 * v + 2 * i], qf[8 * v + 2 * i + 1]),
+                            make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
+        }
         d = (s2.x + s2.y) * pow2i(-C::kE);
       }
       part[j] = d;
@@ -219,14 +275,18 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qf, c
   } else {
 #pragma unroll
     for (int j = 0; j < TPL; ++j) {
-      const uint4* kp = reinterpret_cast<const uint4*>(st + ((TS * j) >> 4) * LOAD + R::kBfK +
-                                                       (r + ((TS * j) & 15)) * D * 2 + 32 * k);
-      const uint4 a = kp[0], c = kp[1];
-      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+      const uint4* kp = reinterpret_cast<const uint4*>(st + ((TS * j) >> 4) * HALF + R::kBfK +
+                                                       (r + ((TS * j) & 15)) * D * 2 + 2 * CW * k);
       float2 s2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        s2 = __ffma2_rn(make_float2(qf[2 * i], qf[2 * i + 1]), make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
+      for (int v = 0; v < CW / 8; ++v) {
+        const uint4 a = kp[v];
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          s2 = __ffma2_rn(make_float2(qfr[8 * v + 2 * i], qfr[8 * v + 2 * i + 1]),
+                          make_float2(bf16_lo(w[i]), bf16_hi(w[i])), s2);
+      }
       part[j] = s2.x + s2.y;
     }
   }
@@ -249,7 +309,7 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qf, c
     ws.l *= c;
     ws.beta *= c;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) ws.acc[i] = __fmul2_rn(ws.acc[i], make_float2(c, c));
+    for (int i = 0; i < CW / 2; ++i) ws.acc[i] = __fmul2_rn(ws.acc[i], make_float2(c, c));
     ws.m = gm;
   }
   // weights carry 2^kVSh (undone once at the end)
@@ -272,32 +332,37 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qf, c
 #pragma unroll
   for (int j = 0; j < TPL; ++j) {
     if constexpr (C::kQuant) {
-      const uint8_t* row = rowbase + tok_off(j);
       const uint32_t mv = *reinterpret_cast<const uint32_t*>(
-          st + ((TS * j) >> 4) * LOAD + R::kVMetaOff +
-          ((r + ((TS * j) & 15)) * (D / kGroup) + (k >> 1)) * 4);
+          st + ((TS * j) >> 4) * HALF + R::kVMetaOff +
+          ((r + ((TS * j) & 15)) * (D / kGroup) + (CW * k) / kGroup) * 4);
       float s = bf16_lo(mv), mn = bf16_hi(mv);
       if (TAIL && tok0 + r + TS * j >= nn) s = mn = 0.f;
-      const uint32_t vh = *reinterpret_cast<const uint32_t*>(row + R::kVHi);
+      uint32_t vh[NWRD], vl[NWRD];
+      plane_words(j, R::kVHi, vh);
+      const float wsc = wgt[j] * s;
+      const float2 ww = make_float2(wsc, wsc);
       if constexpr (C::kFourV) {
-        const uint32_t vl = *reinterpret_cast<const uint32_t*>(row + R::kQ4VLo);
+        plane_words(j, R::kQ4VLo, vl);
         ws.beta = fmaf(wgt[j], mn, ws.beta);
-        axpy16<true>(ws.acc, wgt[j] * s, vh, vl);
-      } else if constexpr (C::kQ4) {
-        ws.beta = fmaf(wgt[j], fmaf(1.5f, s, mn), ws.beta);
-        axpy16<false>(ws.acc, wgt[j] * s, vh, 0u);
+#pragma unroll
+        for (int u = 0; u < NWRD; ++u) axpy16<true>(ws.acc + 8 * u, ww, vh[u], vl[u]);
       } else {
-        ws.beta = fmaf(wgt[j], mn, ws.beta);
-        axpy16<false>(ws.acc, wgt[j] * s, vh, 0u);
+        ws.beta = fmaf(wgt[j], C::kQ4 ? fmaf(1.5f, s, mn) : mn, ws.beta);
+#pragma unroll
+        for (int u = 0; u < NWRD; ++u) axpy16<false>(ws.acc + 8 * u, ww, vh[u], 0u);
       }
     } else {
-      const uint4* vp = reinterpret_cast<const uint4*>(st + ((TS * j) >> 4) * LOAD + R::kBfV +
-                                                       (r + ((TS * j) & 15)) * D * 2 + 32 * k);
-      const uint4 a = vp[0], c = vp[1];
-      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+      const uint4* vp = reinterpret_cast<const uint4*>(st + ((TS * j) >> 4) * HALF + R::kBfV +
+                                                       (r + ((TS * j) & 15)) * D * 2 + 2 * CW * k);
       const float2 ww = make_float2(wgt[j], wgt[j]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ws.acc[i] = __ffma2_rn(ww, make_float2(bf16_lo(w[i]), bf16_hi(w[i])), ws.acc[i]);
+      for (int v = 0; v < CW / 8; ++v) {
+        const uint4 a = vp[v];
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          ws.acc[4 * v + i] = __ffma2_rn(ww, make_float2(bf16_lo(w[i]), bf16_hi(w[i])), ws.acc[4 * v + i]);
+      }
     }
   }
 }
@@ -306,16 +371,18 @@ template <int KIND, int D, bool FULLV, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams p) {
   using C = Cfg<KIND, D, FULLV>;
   using R = typename C::R;
-  constexpr int CH = C::kCH, TS = C::kTS, NSW = C::kNSW;
+  constexpr int CH = C::kCH, CW = C::kCW, NWRD = C::kNWRD, TS = C::kTS, NSW = C::kNSW;
   constexpr int LOAD = C::kLoad, STAGE = C::kStage;
 
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem sp = smem_plan(STAGE, NSW, p.chunk_groups, D, C::kLogits);
   float* logits = reinterpret_cast<float*>(smem + sp.logits);
-  float* wscr = reinterpret_cast<float*>(smem + sp.wscr);
-  float* cta_acc = reinterpret_cast<float*>(smem + sp.cta);
-  float* cta_f = cta_acc + D;
+  auto wscr_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w); };
+  float* cta_acc = reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * 1 + 1024);
+  float* cta_f = reinterpret_cast<float*>(smem + sp.scal);
   int* cta_i = reinterpret_cast<int*>(cta_f);
+  static_assert((D + 4) * 4 <= 1024 && 1024 + D * 4 <= 2 * Cfg<KIND, D, FULLV>::kStage,
+                "result scratch must fit in an idle ring");
 
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int S = gridDim.x;
@@ -338,24 +405,25 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
   // this warp's ring and barriers
   uint8_t* ring = smem + sp.rings + static_cast<size_t>(warp) * NSW * STAGE;
   const uint32_t bar0 = smem_addr(smem + sp.bars) + 8 * NSW * warp;
-  if (lane == 0)
+  if (lane == 0) {
     for (int i = 0; i < NSW; ++i) mbar_init(bar0 + 8 * i, 1);
+    fence_mbar_init();
+  }
   if (threadIdx.x == 0) {
     cta_f[kSlotM] = -INFINITY;
     cta_f[kSlotL] = 0.f;
     cta_i[kSlotCount] = 0;
     cta_i[kSlotBad] = bad;
   }
-  fence_mbar_init();
   __syncthreads();
 
   const int k = lane % CH, r = lane / CH;
-  WarpState ws;
+  WarpState<CW> ws;
   ws.m = -INFINITY;
   ws.l = 0.f;
   ws.beta = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) ws.acc[i] = make_float2(0.f, 0.f);
+  for (int i = 0; i < CW / 2; ++i) ws.acc[i] = make_float2(0.f, 0.f);
 
   // groups of this warp: gi = warp + kNW * it
   const int nit = (!bad && cg > warp) ? (cg - warp + kNW - 1) / kNW : 0;
@@ -378,13 +446,16 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
     }
     return id;
   };
-  int ids = load_ids(0), ids_base = 0;
+  // current and next batch of 16 iterations' ids: the next batch is loaded a
+  // whole batch ahead, so its latency never stalls the ring
+  int ids = load_ids(0), ids_next = load_ids(16), ids_base = 0;
   // issue the bulk copies of iteration `it` into its stage (all lanes call)
   auto issue = [&](int it) {
     if (it >= nit) return;
     if (it - ids_base >= 16) {
       ids_base += 16;
-      ids = load_ids(ids_base);
+      ids = ids_next;
+      ids_next = load_ids(ids_base + 16);
     }
     const int id0 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base));
     const int id1 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base) + 1);
@@ -397,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
       if (id0 >= 0)
         bulk_load(dst, p.arena + (static_cast<size_t>(id0) * p.H + h) * R::kBytes, LOAD, bar, pol);
       if (id1 >= 0)
-        bulk_load(dst + LOAD, p.arena + (static_cast<size_t>(id1) * p.H + h) * R::kBytes, LOAD, bar, pol);
+        bulk_load(dst + C::kHalf, p.arena + (static_cast<size_t>(id1) * p.H + h) * R::kBytes, LOAD, bar, pol);
     }
   };
 
@@ -408,19 +479,23 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
     pdl_wait_prior_grid();  // q, the residual and the newest group may come from the previous kernel
     while (issued < NSW) issue(issued++);
 
-    // this lane's 16 query channels, in log2 units
-    float qf[16], qs[16];
-    {
-      const uint4* qp = reinterpret_cast<const uint4*>(p.q + (static_cast<size_t>(b) * p.H + h) * D + 16 * k);
-      const uint4 a = qp[0], c = qp[1];
-      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+    // query constants (log2 units): qf_c, and qs_c = qf_c * 2^(149 - pos - E)
+    // for the subnormal code views; both in shared memory for all warps
+    float* qconst = reinterpret_cast<float*>(smem + sp.qconst);
+    float* q2buf = reinterpret_cast<float*>(smem + sp.q2buf) + warp * 128;
+    for (int c = lane; c < D; c += 32) {
+      const float qv = __bfloat162float(p.q[(static_cast<size_t>(b) * p.H + h) * D + c]) * p.sm_scale_log2;
+      const int i = c & 15;
+      // every warp writes the same values: no cross-warp ordering is needed
+      qconst[c] = qv;
+      qconst[D + c] = qv * pow2i(149 - (C::kQ4 ? pos4(i) : pos2(i)) - C::kE);
+    }
+    __syncwarp();
+    // bf16 cells keep this lane's query channels in registers
+    float qfr[C::kQuant ? 1 : CW];
+    if constexpr (!C::kQuant) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        qf[2 * i] = bf16_lo(w[i]) * p.sm_scale_log2;
-        qf[2 * i + 1] = bf16_hi(w[i]) * p.sm_scale_log2;
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) qs[i] = qf[i] * pow2i(149 - (C::kQ4 ? pos4(i) : pos2(i)) - C::kE);
+      for (int i = 0; i < CW; ++i) qfr[i] = qconst[CW * k + i];
     }
     const __nv_bfloat16* res = C::kQuant ? p.residual + (static_cast<size_t>(b) * p.H + h) * kGroup * D : nullptr;
 
@@ -435,11 +510,12 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
       const uint8_t* st = ring + stage * STAGE;
       float* lg = logits + gi * kGroup;
       if (tok0 + kGroup <= nn)
-        group_step<KIND, D, FULLV, false>(st, qf, qs, res, tok0, nn, r, k, lg, ws);
+        group_step<KIND, D, FULLV, false>(st, qconst, q2buf, qfr, res, tok0, nn, lane, r, k, lg, ws);
       else
-        group_step<KIND, D, FULLV, true>(st, qf, qs, res, tok0, nn, r, k, lg, ws);
+        group_step<KIND, D, FULLV, true>(st, qconst, q2buf, qfr, res, tok0, nn, lane, r, k, lg, ws);
+      // every shared-memory read of this stage has been consumed above, so
+      // the stage can be refilled
       __syncwarp();
-      if (lane == 0) fence_proxy_async_smem();
       issue(it + NSW);
     }
   }
@@ -448,12 +524,12 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
   // ---- warp results: true per-channel sums, reduced over token sub-groups
   {
     const float unsh = pow2i(-C::kVSh);
-    float o[16];
+    float o[CW];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < CW / 2; ++i) {
       if constexpr (C::kQuant) {
-        const int pa = C::kFourV ? pos4(2 * i) : pos2(2 * i);
-        const int pb = C::kFourV ? pos4(2 * i + 1) : pos2(2 * i + 1);
+        const int pa = C::kFourV ? pos4((2 * i) & 15) : pos2((2 * i) & 15);
+        const int pb = C::kFourV ? pos4((2 * i + 1) & 15) : pos2((2 * i + 1) & 15);
         o[2 * i] = fmaf(ws.acc[i].x, pow2i(64 - pa), ws.beta * unsh);
         o[2 * i + 1] = fmaf(ws.acc[i].y, pow2i(64 - pb), ws.beta * unsh);
       } else {
@@ -465,13 +541,13 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
 #pragma unroll
     for (int off = CH; off < 32; off <<= 1) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) o[i] += __shfl_xor_sync(0xffffffffu, o[i], off);
+      for (int i = 0; i < CW; ++i) o[i] += __shfl_xor_sync(0xffffffffu, o[i], off);
       l += __shfl_xor_sync(0xffffffffu, l, off);
     }
-    float* wsc = wscr + warp * (D + 4);
+    float* wsc = wscr_of(warp);
     if (r == 0) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) wsc[16 * k + i] = o[i];
+      for (int i = 0; i < CW; ++i) wsc[CW * k + i] = o[i];
     }
     if (lane == 0) {
       wsc[D] = ws.m;
@@ -483,13 +559,13 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
   {
     float m_c = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kNW; ++w) m_c = fmaxf(m_c, wscr[w * (D + 4) + D]);
+    for (int w = 0; w < kNW; ++w) m_c = fmaxf(m_c, wscr_of(w)[D]);
     if (threadIdx.x < D) {
       float a = 0.f;
 #pragma unroll
       for (int w = 0; w < kNW; ++w) {
-        const float mw = wscr[w * (D + 4) + D];
-        if (mw != -INFINITY) a = fmaf(fast_exp2(mw - m_c), wscr[w * (D + 4) + threadIdx.x], a);
+        const float mw = wscr_of(w)[D];
+        if (mw != -INFINITY) a = fmaf(fast_exp2(mw - m_c), wscr_of(w)[threadIdx.x], a);
       }
       cta_acc[threadIdx.x] = a;
     }
@@ -497,8 +573,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
       float l = 0.f;
 #pragma unroll
       for (int w = 0; w < kNW; ++w) {
-        const float mw = wscr[w * (D + 4) + D];
-        if (mw != -INFINITY) l = fmaf(fast_exp2(mw - m_c), wscr[w * (D + 4) + D + 1], l);
+        const float mw = wscr_of(w)[D];
+        if (mw != -INFINITY) l = fmaf(fast_exp2(mw - m_c), wscr_of(w)[D + 1], l);
       }
       cta_f[kSlotM] = m_c;
       cta_f[kSlotL] = l;
@@ -540,9 +616,9 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
   const bool want_mask = p.sel_mask != nullptr || p.sel_count != nullptr;
   if (live && ((C::kLogits && p.tau < INFINITY) || want_mask)) {
     const float m_c = cta_f[kSlotM];
-    float corr[16];
+    float corr[CW];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) corr[i] = 0.f;
+    for (int i = 0; i < CW; ++i) corr[i] = 0.f;
     int cnt = 0;
     for (int gi = warp; gi < cg; gi += kNW) {
       const bool valid = (g0 + gi) * kGroup + lane < nn;
@@ -559,6 +635,8 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
         p.sel_mask[(static_cast<size_t>(b) * p.H + h) * p.mask_words + g0 + gi] = mask;
       cnt += __popc(mask);
       if constexpr (C::kLogits) {
+        // up to TS selected tokens at a time: lane (r, k) gathers slot r's
+        // low-plane words of its CW channels
         const int nsel = __popc(mask);
         for (int base = 0; base < nsel; base += TS) {
           const int my = base + r;
@@ -569,12 +647,17 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
           if (my < nsel) {
             const int phys = p.block_table[static_cast<size_t>(b) * p.max_blocks + 2 * (g0 + gi) + (t >> 4)];
             const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
-            const uint32_t lo = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VLo + (t & 15) * R::kRow + 4 * k);
-            const uint32_t mv = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VMeta + ((t & 15) * (D / kGroup) + (k >> 1)) * 4);
+            const uint32_t mv = *reinterpret_cast<const uint32_t*>(
+                rec + R::kQ4VMeta + ((t & 15) * (D / kGroup) + (CW * k) / kGroup) * 4);
             const float wsel = fast_exp2(lt - m_c) * bf16_lo(mv);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              corr[i] = fmaf(wsel, static_cast<float>((lo >> (2 * i)) & 3u) - 1.5f, corr[i]);
+            for (int u = 0; u < NWRD; ++u) {
+              const uint32_t lo = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VLo + (t & 15) * R::kRow +
+                                                                   4 * (NWRD * k + u));
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                corr[16 * u + i] = fmaf(wsel, static_cast<float>((lo >> (2 * i)) & 3u) - 1.5f, corr[16 * u + i]);
+            }
           }
         }
       }
@@ -583,10 +666,10 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
 #pragma unroll
       for (int off = CH; off < 32; off <<= 1)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) corr[i] += __shfl_xor_sync(0xffffffffu, corr[i], off);
+        for (int i = 0; i < CW; ++i) corr[i] += __shfl_xor_sync(0xffffffffu, corr[i], off);
       if (r == 0) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) atomicAdd(&cta_acc[16 * k + i], corr[i]);
+        for (int i = 0; i < CW; ++i) atomicAdd(&cta_acc[CW * k + i], corr[i]);
       }
     }
     if (lane == 0) atomicAdd(&cta_i[kSlotCount], cnt);
@@ -636,16 +719,34 @@ size_t smem_bytes_t(int cg) {
   return smem_plan(C::kStage, C::kNSW, cg, D, C::kLogits).total;
 }
 
+// CTAs of this instantiation that can be resident at once on the device
+// (for clusters: co-resident clusters times the cluster size).
 template <int KIND, int D, bool FULLV, bool CLUSTER>
-int occupancy_t(int cg) {
-  int blocks = 0;
+long resident_ctas_t(int cg, int splits, int sms) {
   const size_t smem = smem_bytes_t<KIND, D, FULLV, CLUSTER>(cg);
   if (smem > 227u * 1024u) return 0;
   auto kern = decode_kernel<KIND, D, FULLV, CLUSTER>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kThreads, smem) != cudaSuccess) return 0;
-  return blocks;
+  if (!CLUSTER) {
+    int blocks = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kThreads, smem) != cudaSuccess) return 0;
+    return static_cast<long>(blocks) * sms;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(splits, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = splits;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return 0;
+  return static_cast<long>(clusters) * splits;
 }
 
 template <int KIND, int D, bool FULLV, bool CLUSTER>
@@ -686,19 +787,20 @@ cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t 
 }
 
 template <int KIND, int D, bool FULLV>
-int occupancy_c(bool cluster, int cg) {
-  return cluster ? occupancy_t<KIND, D, FULLV, true>(cg) : occupancy_t<KIND, D, FULLV, false>(cg);
+long resident_c(int cg, int splits, int sms) {
+  return splits > 1 ? resident_ctas_t<KIND, D, FULLV, true>(cg, splits, sms)
+                    : resident_ctas_t<KIND, D, FULLV, false>(cg, splits, sms);
 }
 
-// CTAs of one decode instantiation that fit on one SM.
-int blocks_per_sm(int kind, int d, bool cluster, int cg) {
+// Co-resident CTAs of one decode instantiation (0 without a device).
+long resident_ctas(int kind, int d, int cg, int splits, int sms) {
   switch (kind * 1000 + d) {
-    case LOOPKV_CELL_Q4 * 1000 + 128: return occupancy_c<LOOPKV_CELL_Q4, 128, false>(cluster, cg);
-    case LOOPKV_CELL_Q4 * 1000 + 64: return occupancy_c<LOOPKV_CELL_Q4, 64, false>(cluster, cg);
-    case LOOPKV_CELL_Q2 * 1000 + 128: return occupancy_c<LOOPKV_CELL_Q2, 128, false>(cluster, cg);
-    case LOOPKV_CELL_Q2 * 1000 + 64: return occupancy_c<LOOPKV_CELL_Q2, 64, false>(cluster, cg);
-    case LOOPKV_CELL_BF16 * 1000 + 128: return occupancy_c<LOOPKV_CELL_BF16, 128, false>(cluster, cg);
-    case LOOPKV_CELL_BF16 * 1000 + 64: return occupancy_c<LOOPKV_CELL_BF16, 64, false>(cluster, cg);
+    case LOOPKV_CELL_Q4 * 1000 + 128: return resident_c<LOOPKV_CELL_Q4, 128, false>(cg, splits, sms);
+    case LOOPKV_CELL_Q4 * 1000 + 64: return resident_c<LOOPKV_CELL_Q4, 64, false>(cg, splits, sms);
+    case LOOPKV_CELL_Q2 * 1000 + 128: return resident_c<LOOPKV_CELL_Q2, 128, false>(cg, splits, sms);
+    case LOOPKV_CELL_Q2 * 1000 + 64: return resident_c<LOOPKV_CELL_Q2, 64, false>(cg, splits, sms);
+    case LOOPKV_CELL_BF16 * 1000 + 128: return resident_c<LOOPKV_CELL_BF16, 128, false>(cg, splits, sms);
+    case LOOPKV_CELL_BF16 * 1000 + 64: return resident_c<LOOPKV_CELL_BF16, 64, false>(cg, splits, sms);
     default: return 0;
   }
 }
@@ -721,9 +823,8 @@ int decode_splits(int kind, int head_dim, int batch, int heads, int max_seq_len)
   for (int s = min_s; s <= 8; s <<= 1) {
     if (s > min_s && groups < 2 * kNW * s) break;  // keep >= 2 groups per warp
     const int cg = (groups + s - 1) / s;
-    int per_sm = blocks_per_sm(kind, head_dim, s > 1, cg);
-    if (per_sm <= 0) per_sm = 4;  // no device: a fixed guess keeps the choice deterministic
-    const long slots = static_cast<long>(sms) * per_sm;
+    long slots = resident_ctas(kind, head_dim, cg, s, sms);
+    if (slots <= 0) slots = 4L * sms;  // no device: a fixed guess keeps the choice deterministic
     const long ctas = pairs * s;
     const long waves = (ctas + slots - 1) / slots;
     const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);

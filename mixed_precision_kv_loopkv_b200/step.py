@@ -22,6 +22,22 @@ from .loopkv import (LOOPKV_CELL_REUSE, KVCells, loopkv_decode_attention,
                      loopkv_quantize_append)
 
 
+def prefill(kv: KVCells, loop: int, layer: int, k, v, block_table, lens, err_flag=None, stream=None):
+    """Append the first lens[b] tokens of k, v (bf16 [B, n_max, H, D]) to the
+    cell, sequences of different lengths included: one append per distinct
+    length, sequences already complete skipped (negative start position)."""
+    lens = [int(x) for x in (lens.tolist() if hasattr(lens, "tolist") else lens)]
+    prev = 0
+    for cut in sorted(set(lens)):
+        if cut <= prev:
+            continue
+        starts = [prev if n >= cut else -1 for n in lens]
+        pos = torch.tensor(starts, dtype=torch.int32, device=k.device)
+        loopkv_quantize_append(kv, loop, layer, k[:, prev:cut].contiguous(), v[:, prev:cut].contiguous(),
+                               block_table, pos, err_flag=err_flag, stream=stream)
+        prev = cut
+
+
 class LoopedDecodeStep:
     """Sequences the per-cell kernels of one decode step (graph-capturable).
 

@@ -24,7 +24,7 @@ def build_store(w, cells=None, capacity=None, device="cuda", flags=0, splits=0, 
     need their final-loop source).  Returns (kv, plan, table, lens, kvdata)
     with kvdata[cell] = (K, V) bf16 [B, n_max, H, D] on the device.
     """
-    from mixed_precision_kv_loopkv_b200 import KVCells, loopkv_quantize_append
+    from mixed_precision_kv_loopkv_b200 import KVCells, prefill as prefill_cell
 
     plan = make_plan(w)
     lens = seq_lens_for(w)
@@ -39,16 +39,17 @@ def build_store(w, cells=None, capacity=None, device="cuda", flags=0, splits=0, 
                  allocate=want)
     table_d = torch.from_numpy(table).to(device)
     lens_d = torch.from_numpy(lens).to(device)
-    zero = torch.zeros(w.batch, dtype=torch.int32, device=device)
     data = {}
     if prefill:
+        err = torch.zeros(1, dtype=torch.int32, device=device)
         for c in sorted(want):
             if plan[c] == "reuse":
                 continue
             loop, layer = divmod(c, w.num_layers)
             k, v = cell_kv(w, loop, layer, device=device)
-            loopkv_quantize_append(kv, loop, layer, k, v, table_d, zero)
+            prefill_cell(kv, loop, layer, k, v, table_d, lens, err_flag=err)
             data[c] = (k, v)
+        assert int(err) == 0, f"prefill flagged device error {int(err)}"
     return kv, plan, table_d, lens_d, data
 
 
