@@ -50,8 +50,10 @@
  *     kernels never trap;
  *   - the library keeps no global state; concurrent calls on different
  *     streams are safe as long as they do not write the same cells.
- * Inputs must be finite; the fp32 arithmetic assumes |q * scale * sm_scale|
- * and value scales below 2^40.
+ * Inputs must be finite; the fp32 key arithmetic assumes |q * scale * sm_scale|
+ * below 2^40; value scales (max - min of a 32-channel group over 3 or 15) must
+ * not exceed 255 (|values| up to about 750 for 2-bit and 3800 for 4-bit cells):
+ * the append flags larger ones with LOOPKV_DEVERR_RANGE.
  */
 #ifndef LOOPKV_H
 #define LOOPKV_H
@@ -89,6 +91,8 @@ typedef enum {
 #define LOOPKV_DEVERR_BLOCK_ID 0x1 /* block-table entry outside [0, num_blocks) */
 #define LOOPKV_DEVERR_SEQ_LEN 0x2  /* length beyond the block table or max_seq_len */
 #define LOOPKV_DEVERR_TIMEOUT 0x4  /* a bounded wait on the device gave up */
+#define LOOPKV_DEVERR_RANGE 0x8    /* a value group's scale exceeds 255: the decode
+                                      kernel's f16 value weights would overflow */
 
 /* loopkv_config.flags */
 #define LOOPKV_FLAG_PDL 0x1 /* programmatic dependent launch: a kernel may start

@@ -16,6 +16,7 @@ from .loopkv import (  # noqa: F401
     LOOPKV_CELL_Q4,
     LOOPKV_CELL_REUSE,
     LOOPKV_DEVERR_BLOCK_ID,
+    LOOPKV_DEVERR_RANGE,
     LOOPKV_DEVERR_SEQ_LEN,
     LOOPKV_DEVERR_TIMEOUT,
     LOOPKV_FLAG_PDL,

@@ -22,6 +22,9 @@
 namespace loopkv {
 namespace {
 
+// Largest value-group scale the decode kernel's f16 value weights carry.
+constexpr float kMaxValueScale = 255.f;
+
 __device__ __forceinline__ float warp_min(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
@@ -137,9 +140,11 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
         if constexpr (kSplit)
           *reinterpret_cast<uint32_t*>(rec + R::kQ4VLo + row * R::kRow + word * 4) = w_lo;
       }
-      if (lane == 0)
+      if (lane == 0) {
         *reinterpret_cast<uint32_t*>(rec + R::kVMetaOff + (row * kVGroups + g) * 4) =
             meta_word(s_b, mn_b);
+        if (s_b > kMaxValueScale) flag_error(p.err, LOOPKV_DEVERR_RANGE);
+      }
     }
 
     // 2. key groups completed by this call: groups [start/32, end/32 - 1]

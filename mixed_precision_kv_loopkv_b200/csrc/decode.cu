@@ -36,6 +36,8 @@
 
 #include <algorithm>
 
+#include <cuda_fp16.h>
+
 #include "device_common.cuh"
 #include "kernels.h"
 
@@ -112,6 +114,38 @@ __device__ __forceinline__ void axpy16(float2* acc, float2 ww, uint32_t a, uint3
   }
 }
 
+// Mixed-precision FMA: fp32 accumulator += f16 x f16 (low / high half of a
+// 32-bit register times the f16 in the low half of w).  The product of two
+// f16 values is exact in fp32.
+__device__ __forceinline__ float fma_h_lo(uint32_t f, uint32_t w, float c) {
+  float d;
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %3;\n\t}"
+      : "=f"(d) : "r"(f), "r"(w), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fma_h_hi(uint32_t f, uint32_t w, float c) {
+  float d;
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a1, b0, %3;\n\t}"
+      : "=f"(d) : "r"(f), "r"(w), "f"(c));
+  return d;
+}
+// One AND isolates channel i (i < 8) in the low half and channel i + 8 in the
+// high half of a 2-bit plane word, both as f16 subnormals code * 2^(p - 24),
+// p = 2i for i < 5 and 2(i - 5) after a 10-bit shift for the rest.
+__host__ __device__ constexpr int posh(int i) { return 2 * (i < 5 ? i : i - 5); }
+// acc[i] += w * (channel i, channel i + 8) of one 16-channel word; w is f16.
+__device__ __forceinline__ void axpy16_h(float2* acc, uint32_t wh, uint32_t x) {
+  const uint32_t x10 = x >> 10;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t f = i < 5 ? (x & (0x00030003u << (2 * i))) : (x10 & (0x00030003u << (2 * (i - 5))));
+    acc[i].x = fma_h_lo(f, wh, acc[i].x);
+    acc[i].y = fma_h_hi(f, wh, acc[i].y);
+  }
+}
+
 template <int KIND, int D, bool FULLV>
 struct Cfg {
   using R = Rec<KIND, D>;
@@ -130,8 +164,12 @@ struct Cfg {
   static constexpr int kTS = 32 / kCH;                     // token sub-groups per warp
   static constexpr int kTPL = 32 / kTS;                    // tokens per lane per group
   static constexpr int kE = kQuant ? kExpOff : 0;
+  // 2-bit value fields go through f16 x f16 -> fp32 FMAs; the full 4-bit
+  // values of the tau = 0 variant and bf16 cells stay on FP32x2 FMAs
+  static constexpr bool kHalfV = kQuant && !FULLV;
   // power of two folded into the softmax weight for the value products
-  static constexpr int kVSh = !kQuant ? 0 : (kQ4 && !FULLV) ? 87 : 85;
+  // (half path: weights <= 2^6 keep value scales up to 2^9 inside f16)
+  static constexpr int kVSh = !kQuant ? 0 : kHalfV ? 6 : 85;
   static constexpr bool kLogits = kQ4 && !FULLV;           // pass 2 needs the logits
   static constexpr bool kFourV = kQ4 && FULLV;             // full 4-bit values in pass 1
 };
@@ -340,16 +378,18 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
       uint32_t vh[NWRD], vl[NWRD];
       plane_words(j, R::kVHi, vh);
       const float wsc = wgt[j] * s;
-      const float2 ww = make_float2(wsc, wsc);
       if constexpr (C::kFourV) {
+        const float2 ww = make_float2(wsc, wsc);
         plane_words(j, R::kQ4VLo, vl);
         ws.beta = fmaf(wgt[j], mn, ws.beta);
 #pragma unroll
         for (int u = 0; u < NWRD; ++u) axpy16<true>(ws.acc + 8 * u, ww, vh[u], vl[u]);
       } else {
+        // 4-bit high plane: the weight carries the factor 4 of 4*hi
+        const uint32_t wh = __half_as_ushort(__float2half_rn(C::kQ4 ? 4.f * wsc : wsc));
         ws.beta = fmaf(wgt[j], C::kQ4 ? fmaf(1.5f, s, mn) : mn, ws.beta);
 #pragma unroll
-        for (int u = 0; u < NWRD; ++u) axpy16<false>(ws.acc + 8 * u, ww, vh[u], 0u);
+        for (int u = 0; u < NWRD; ++u) axpy16_h(ws.acc + 8 * u, wh, vh[u]);
       }
     } else {
       const uint4* vp = reinterpret_cast<const uint4*>(st + ((TS * j) >> 4) * HALF + R::kBfV +
@@ -527,9 +567,15 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
     float o[CW];
 #pragma unroll
     for (int i = 0; i < CW / 2; ++i) {
-      if constexpr (C::kQuant) {
-        const int pa = C::kFourV ? pos4((2 * i) & 15) : pos2((2 * i) & 15);
-        const int pb = C::kFourV ? pos4((2 * i + 1) & 15) : pos2((2 * i + 1) & 15);
+      if constexpr (C::kHalfV) {
+        // pair i of word u: channels 16u + (i & 7) and 16u + (i & 7) + 8
+        const int u = i >> 3, ii = i & 7;
+        const float sc = pow2i(24 - posh(ii) - C::kVSh);
+        o[16 * u + ii] = fmaf(ws.acc[i].x, sc, ws.beta * unsh);
+        o[16 * u + ii + 8] = fmaf(ws.acc[i].y, sc, ws.beta * unsh);
+      } else if constexpr (C::kQuant) {
+        const int pa = pos4((2 * i) & 15);
+        const int pb = pos4((2 * i + 1) & 15);
         o[2 * i] = fmaf(ws.acc[i].x, pow2i(64 - pa), ws.beta * unsh);
         o[2 * i + 1] = fmaf(ws.acc[i].y, pow2i(64 - pb), ws.beta * unsh);
       } else {

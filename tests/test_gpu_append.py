@@ -120,3 +120,17 @@ def test_append_flags_bad_block_and_overflow():
     loopkv_quantize_append(kv, 0, 0, k, k, table, torch.tensor([20, 0], dtype=torch.int32, device="cuda"),
                            err_flag=err)
     assert int(err) & LOOPKV_DEVERR_SEQ_LEN
+
+
+def test_append_flags_value_scale_out_of_range():
+    from mixed_precision_kv_loopkv_b200 import LOOPKV_DEVERR_RANGE, KVCells, loopkv_quantize_append
+    kv = KVCells(["q4"], 1, 1, 1, 64, 2, 1, 2)
+    table = torch.tensor([[0, 1]], dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    k = torch.randn(1, 4, 1, 64, device="cuda").to(torch.bfloat16)
+    v = k.clone()
+    loopkv_quantize_append(kv, 0, 0, k, v, table, torch.zeros(1, dtype=torch.int32, device="cuda"), err_flag=err)
+    assert int(err) == 0
+    v[0, 3, 0, 7] = 5000.0          # range 5000 / 15 > 255
+    loopkv_quantize_append(kv, 0, 0, k, v, table, torch.zeros(1, dtype=torch.int32, device="cuda"), err_flag=err)
+    assert int(err) & LOOPKV_DEVERR_RANGE
