@@ -175,12 +175,17 @@ struct Cfg {
 };
 
 // Shared-memory carve-up (bytes), identical on host and device.
-// After pass 1 a warp's ring is idle: its result scratch (wscr) lives at the
-// start of its own ring, and the CTA accumulators (used after a CTA barrier)
-// in warp 1's ring past that warp's scratch.
+// After pass 1 a warp's ring is idle and holds the warp's results: its
+// per-channel sums (wscr, at the ring's start) and its low-plane corrections
+// (at +kCorrOff).  The exchange area (xchg) is never aliased: peers of the
+// cluster store into it while this CTA may still be in pass 1.
+//   xchg: table float4[8 * kNW] (every warp's max, sum, error bits),
+//         red float[D] (the owner's slice sums of every split),
+//         cnts int32[8] (every split's selection count)
 struct Smem {
-  size_t rings, ring_bytes, bars, qconst, q2buf, logits, scal, total;
+  size_t rings, ring_bytes, bars, qconst, q2buf, logits, ids, masks, xchg, scal, total;
 };
+constexpr int kCorrOff = 1024;
 __host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int d, bool logits) {
   Smem s;
   s.rings = 0;
@@ -189,13 +194,17 @@ __host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int 
   s.qconst = s.bars + 8 * nsw * kNW;                       // qf[D], qs[D]
   s.q2buf = s.qconst + static_cast<size_t>(8) * d;         // per warp: 128 floats, swizzled
   s.logits = s.q2buf + static_cast<size_t>(4) * 128 * kNW;
-  s.scal = s.logits + (logits ? 128 * static_cast<size_t>(cg) : 0);  // CTA scalars
-  s.total = s.scal + 16;
+  s.ids = s.logits + (logits ? 128 * static_cast<size_t>(cg) : 0);  // two block ids per group
+  s.masks = s.ids + (logits ? 8 * static_cast<size_t>(cg) : 0);     // selection word per group
+  s.xchg = s.masks + (logits ? 4 * static_cast<size_t>(cg) : 0);
+  s.xchg = (s.xchg + 15) & ~static_cast<size_t>(15);
+  s.scal = s.xchg + 16 * 8 * kNW + 4 * static_cast<size_t>(d) + 32;  // CTA scalars, warp counts
+  s.total = s.scal + 32;
   return s;
 }
 
-// Per-CTA scalar slots in the cta segment after the D accumulators.
-enum { kSlotM = 0, kSlotL = 1, kSlotCount = 2, kSlotBad = 3 };
+// Per-CTA scalar slots.
+enum { kSlotBad = 0, kSlotCnt0 = 4 };
 
 // Per-lane running state of one warp's online softmax.
 template <int CW>
@@ -418,11 +427,14 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
   const Smem sp = smem_plan(STAGE, NSW, p.chunk_groups, D, C::kLogits);
   float* logits = reinterpret_cast<float*>(smem + sp.logits);
   auto wscr_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w); };
-  float* cta_acc = reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * 1 + 1024);
-  float* cta_f = reinterpret_cast<float*>(smem + sp.scal);
-  int* cta_i = reinterpret_cast<int*>(cta_f);
-  static_assert((D + 4) * 4 <= 1024 && 1024 + D * 4 <= 2 * Cfg<KIND, D, FULLV>::kStage,
-                "result scratch must fit in an idle ring");
+  auto corr_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w + kCorrOff); };
+  int32_t* ids_smem = reinterpret_cast<int32_t*>(smem + sp.ids);
+  uint32_t* masks_smem = reinterpret_cast<uint32_t*>(smem + sp.masks);
+  float4* table = reinterpret_cast<float4*>(smem + sp.xchg);
+  float* red = reinterpret_cast<float*>(smem + sp.xchg + 16 * 8 * kNW);
+  int* cnts = reinterpret_cast<int*>(smem + sp.xchg + 16 * 8 * kNW + 4 * D);
+  int* cta_i = reinterpret_cast<int*>(smem + sp.scal);
+  static_assert(D * 4 <= kCorrOff && kCorrOff + D * 4 <= NSW * STAGE, "warp results must fit in an idle ring");
 
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int S = gridDim.x;
@@ -449,13 +461,9 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
     for (int i = 0; i < NSW; ++i) mbar_init(bar0 + 8 * i, 1);
     fence_mbar_init();
   }
-  if (threadIdx.x == 0) {
-    cta_f[kSlotM] = -INFINITY;
-    cta_f[kSlotL] = 0.f;
-    cta_i[kSlotCount] = 0;
-    cta_i[kSlotBad] = bad;
-  }
+  if (threadIdx.x == 0) cta_i[kSlotBad] = bad;
   __syncthreads();
+  if constexpr (CLUSTER) cluster_arrive_relaxed();
 
   const int k = lane % CH, r = lane / CH;
   WarpState<CW> ws;
@@ -469,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
   const int nit = (!bad && cg > warp) ? (cg - warp + kNW - 1) / kNW : 0;
   const int g_unsafe = (nn - 1) / kGroup;  // may be written by the previous kernel
   const uint64_t pol = l2_evict_first_policy();
-  const int32_t* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+  const int32_t* btab = p.block_table + static_cast<size_t>(b) * p.max_blocks;
   // block ids of 16 iterations, two per iteration, spread over the lanes
   auto load_ids = [&](int it0) {
     const int it = it0 + (lane >> 1);
@@ -477,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
     if (it < nit) {
       const int lb = 2 * (g0 + warp + kNW * it) + (lane & 1);
       if (lb < n_blocks) {
-        id = table[lb];
+        id = btab[lb];
         if (id < 0 || id >= p.num_blocks) {
           atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_BLOCK_ID);
           id = -1;
@@ -499,6 +507,10 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
     }
     const int id0 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base));
     const int id1 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base) + 1);
+    if (C::kLogits && lane == 0) {  // kept for the low-plane gather of pass 2
+      ids_smem[2 * (warp + kNW * it)] = id0;
+      ids_smem[2 * (warp + kNW * it) + 1] = id1;
+    }
     if (lane == 0) {
       const int stage = it % NSW;
       const uint32_t bar = bar0 + 8 * stage;
@@ -561,7 +573,9 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
   }
   pdl_wait_prior_grid();  // nothing below may run ahead of the previous kernel
 
-  // ---- warp results: true per-channel sums, reduced over token sub-groups
+  // ---- this warp's result in its own scale 2^-m_w: true per-channel sums,
+  //      reduced over the token sub-groups
+  float lw;
   {
     const float unsh = pow2i(-C::kVSh);
     float o[CW];
@@ -583,180 +597,206 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
         o[2 * i + 1] = ws.acc[i].y;
       }
     }
-    float l = ws.l * unsh;
+    lw = ws.l * unsh;
 #pragma unroll
     for (int off = CH; off < 32; off <<= 1) {
 #pragma unroll
       for (int i = 0; i < CW; ++i) o[i] += __shfl_xor_sync(0xffffffffu, o[i], off);
-      l += __shfl_xor_sync(0xffffffffu, l, off);
+      lw += __shfl_xor_sync(0xffffffffu, lw, off);
     }
     float* wsc = wscr_of(warp);
     if (r == 0) {
 #pragma unroll
       for (int i = 0; i < CW; ++i) wsc[CW * k + i] = o[i];
     }
-    if (lane == 0) {
-      wsc[D] = ws.m;
-      wsc[D + 1] = l;
-    }
   }
-  __syncthreads();
-  // ---- CTA merge (CTA-local scale m_cta)
-  {
-    float m_c = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kNW; ++w) m_c = fmaxf(m_c, wscr_of(w)[D]);
-    if (threadIdx.x < D) {
-      float a = 0.f;
-#pragma unroll
-      for (int w = 0; w < kNW; ++w) {
-        const float mw = wscr_of(w)[D];
-        if (mw != -INFINITY) a = fmaf(fast_exp2(mw - m_c), wscr_of(w)[threadIdx.x], a);
-      }
-      cta_acc[threadIdx.x] = a;
-    }
-    if (threadIdx.x == 0) {
-      float l = 0.f;
-#pragma unroll
-      for (int w = 0; w < kNW; ++w) {
-        const float mw = wscr_of(w)[D];
-        if (mw != -INFINITY) l = fmaf(fast_exp2(mw - m_c), wscr_of(w)[D + 1], l);
-      }
-      cta_f[kSlotM] = m_c;
-      cta_f[kSlotL] = l;
-    }
-  }
-  if constexpr (CLUSTER) cluster_sync_all(); else __syncthreads();
 
-  // ---- global (max, normaliser) over the splits
-  float m_g = -INFINITY, z = 0.f;
-  int any_bad = 0;
-  const uint32_t my_f = smem_addr(cta_f);
-  for (int s = 0; s < S; ++s) {
-    float ms, ls;
-    int bs;
+  // ---- publish (max, sum, error bits) of this warp into every split's table
+  //      (the error word includes this warp's own flags, set before this read)
+  if constexpr (CLUSTER) cluster_wait();  // every CTA of the cluster has started
+  {
+    const float4 ent = make_float4(ws.m, lw, __int_as_float(cta_i[kSlotBad]), 0.f);
+    const int e = split * kNW + warp;
     if constexpr (CLUSTER) {
-      const uint32_t pa = peer_addr(my_f, s);
-      ms = ld_peer_f32(pa + 4 * kSlotM);
-      ls = ld_peer_f32(pa + 4 * kSlotL);
-      bs = ld_peer_s32(pa + 4 * kSlotBad);
-    } else {
-      ms = cta_f[kSlotM];
-      ls = cta_f[kSlotL];
-      bs = cta_i[kSlotBad];
+      if (lane < S) st_peer_v4(peer_addr(smem_addr(table + e), lane), ent);
+    } else if (lane == 0) {
+      table[e] = ent;
     }
-    any_bad |= bs;
-    if (ms != -INFINITY) {
-      if (ms > m_g) {
-        z = z * fast_exp2(m_g - ms) + ls;
-        m_g = ms;
-      } else {
-        z = fmaf(ls, fast_exp2(ms - m_g), z);
+  }
+  if constexpr (CLUSTER) cluster_arrive_release();
+
+  // ---- while the splits meet: bring the low-plane rows of this warp's
+  //      candidates into L2.  A token's weight under the global normaliser is
+  //      at most its weight under this warp's own (max, sum), so every token
+  //      pass 2 selects is among these.
+  if (C::kLogits && p.tau > 0.f && p.tau < INFINITY && lw > 0.f) {
+    const float thr = p.tau * lw;
+    for (int gi = warp; gi < cg; gi += kNW) {
+      const float lg = logits[gi * kGroup + lane];
+      if ((g0 + gi) * kGroup + lane < nn && fast_exp2(lg - ws.m) >= thr) {
+        const int phys = ids_smem[2 * gi + (lane >> 4)];
+        if (phys >= 0) {
+          const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
+          prefetch_l2(rec + R::kQ4VLo + (lane & 15) * R::kRow);
+          prefetch_l2(rec + R::kQ4VMeta + (lane & 15) * (D / kGroup) * 4);
+        }
       }
     }
+  }
+  if constexpr (CLUSTER) cluster_wait_acquire(); else __syncthreads();
+
+  // ---- global (max, normaliser, errors) from the local table
+  float m_g, z;
+  int any_bad;
+  {
+    float me = -INFINITY, le = 0.f;
+    int be = 0;
+    if (lane < S * kNW) {
+      const float4 t = table[lane];
+      me = t.x;
+      le = t.y;
+      be = __float_as_int(t.z);
+    }
+    m_g = me;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m_g = fmaxf(m_g, __shfl_xor_sync(0xffffffffu, m_g, off));
+    z = (me == -INFINITY) ? 0.f : le * fast_exp2(me - m_g);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    any_bad = static_cast<int>(__reduce_or_sync(0xffffffffu, static_cast<unsigned>(be)));
   }
   const bool live = !any_bad && z > 0.f;
   const float inv_z = live ? 1.f / z : 0.f;
 
-  // ---- pass 2: low-plane selection and gather (4-bit sources)
+  // ---- pass 2a: low-plane selection of every group of this warp
   const bool want_mask = p.sel_mask != nullptr || p.sel_count != nullptr;
-  if (live && ((C::kLogits && p.tau < INFINITY) || want_mask)) {
-    const float m_c = cta_f[kSlotM];
-    float corr[CW];
-#pragma unroll
-    for (int i = 0; i < CW; ++i) corr[i] = 0.f;
-    int cnt = 0;
+  const bool gather = C::kLogits && p.tau < INFINITY;
+  int cnt = 0;
+  if (live && (gather || want_mask)) {
     for (int gi = warp; gi < cg; gi += kNW) {
       const bool valid = (g0 + gi) * kGroup + lane < nn;
-      float lg = 0.f;
       bool sel;
       if constexpr (C::kLogits) {
-        lg = logits[gi * kGroup + lane];
-        sel = valid && (fast_exp2(lg - m_g) * inv_z >= p.tau);
+        sel = valid && (fast_exp2(logits[gi * kGroup + lane] - m_g) * inv_z >= p.tau);
       } else {
         sel = C::kQ4 && valid;  // tau = 0: every token took its low plane in pass 1
       }
       const uint32_t mask = __ballot_sync(0xffffffffu, sel);
-      if (p.sel_mask && lane == 0)
-        p.sel_mask[(static_cast<size_t>(b) * p.H + h) * p.mask_words + g0 + gi] = mask;
+      if (lane == 0) {
+        if (p.sel_mask) p.sel_mask[(static_cast<size_t>(b) * p.H + h) * p.mask_words + g0 + gi] = mask;
+        if constexpr (C::kLogits) masks_smem[gi] = mask;
+      }
       cnt += __popc(mask);
-      if constexpr (C::kLogits) {
-        // up to TS selected tokens at a time: lane (r, k) gathers slot r's
-        // low-plane words of its CW channels
-        const int nsel = __popc(mask);
-        for (int base = 0; base < nsel; base += TS) {
-          const int my = base + r;
-          uint32_t mm = mask;
-          for (int q = 0; q < my && mm; ++q) mm &= mm - 1;
-          const int t = (my < nsel) ? (__ffs(mm) - 1) : 0;
-          const float lt = __shfl_sync(0xffffffffu, lg, t);
-          if (my < nsel) {
-            const int phys = p.block_table[static_cast<size_t>(b) * p.max_blocks + 2 * (g0 + gi) + (t >> 4)];
-            const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
-            const uint32_t mv = *reinterpret_cast<const uint32_t*>(
-                rec + R::kQ4VMeta + ((t & 15) * (D / kGroup) + (CW * k) / kGroup) * 4);
-            const float wsel = fast_exp2(lt - m_c) * bf16_lo(mv);
+    }
+  }
+  __syncwarp();  // lane 0's selection words are read by the whole warp below
+
+  // ---- pass 2b: gather the selected tokens' low-plane rows, kNB tokens per
+  //      round trip; lane l owns channels 4l .. 4l + 3 (one byte of the row)
+  //      and adds p * scale * (lo - 1.5) in the final units
+  if constexpr (C::kLogits) {
+    if (live && gather) {
+      constexpr int kNB = 4;
+      float corr[4] = {0.f, 0.f, 0.f, 0.f};
+      int gcur = warp;
+      uint32_t mcur = (cnt > 0 && gcur < cg) ? masks_smem[gcur] : 0u;
+      int left = cnt;
+      while (left > 0) {
+        int tg[kNB], tt[kNB];
 #pragma unroll
-            for (int u = 0; u < NWRD; ++u) {
-              const uint32_t lo = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VLo + (t & 15) * R::kRow +
-                                                                   4 * (NWRD * k + u));
+        for (int j = 0; j < kNB; ++j) {
+          while (mcur == 0u && left > 0 && gcur + kNW < cg) {
+            gcur += kNW;
+            mcur = masks_smem[gcur];
+          }
+          tg[j] = -1;
+          tt[j] = 0;
+          if (mcur != 0u && left > 0) {
+            tg[j] = gcur;
+            tt[j] = __ffs(mcur) - 1;
+            mcur &= mcur - 1u;
+            --left;
+          }
+        }
+        uint32_t mv[kNB], lo[kNB];
+        float lgv[kNB];
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                corr[16 * u + i] = fmaf(wsel, static_cast<float>((lo >> (2 * i)) & 3u) - 1.5f, corr[16 * u + i]);
+        for (int j = 0; j < kNB; ++j) {
+          mv[j] = 0u;
+          lo[j] = 0u;
+          lgv[j] = -INFINITY;
+          if (tg[j] >= 0) {
+            const int phys = ids_smem[2 * tg[j] + (tt[j] >> 4)];
+            lgv[j] = logits[tg[j] * kGroup + tt[j]];
+            if (phys >= 0 && lane < D / 4) {
+              const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
+              mv[j] = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VMeta +
+                                                         ((tt[j] & 15) * (D / kGroup) + (4 * lane) / kGroup) * 4);
+              lo[j] = rec[R::kQ4VLo + (tt[j] & 15) * R::kRow + lane];
             }
           }
         }
+#pragma unroll
+        for (int j = 0; j < kNB; ++j) {
+          const float wsel = fast_exp2(lgv[j] - m_g) * inv_z * bf16_lo(mv[j]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            corr[i] = fmaf(wsel, static_cast<float>((lo[j] >> (2 * i)) & 3u) - 1.5f, corr[i]);
+        }
       }
+      if (lane < D / 4)
+        *reinterpret_cast<float4*>(corr_of(warp) + 4 * lane) = make_float4(corr[0], corr[1], corr[2], corr[3]);
     }
-    if constexpr (C::kLogits) {
-#pragma unroll
-      for (int off = CH; off < 32; off <<= 1)
-#pragma unroll
-        for (int i = 0; i < CW; ++i) corr[i] += __shfl_xor_sync(0xffffffffu, corr[i], off);
-      if (r == 0) {
-#pragma unroll
-        for (int i = 0; i < CW; ++i) atomicAdd(&cta_acc[CW * k + i], corr[i]);
-      }
-    }
-    if (lane == 0) atomicAdd(&cta_i[kSlotCount], cnt);
   }
-  if constexpr (CLUSTER) cluster_sync_all(); else __syncthreads();
+  if (lane == 0) cta_i[kSlotCnt0 + warp] = cnt;
+  __syncthreads();  // every warp's sums, corrections and counts are in shared memory
 
-  // ---- combine the splits; rank s writes channels [s*D/S, (s+1)*D/S)
+  // ---- push this CTA's share of every channel, in the final units, to the
+  //      split that owns the channel: rank s owns [s*D/S, (s+1)*D/S)
   const int per_rank = D / S;
-  if (threadIdx.x < per_rank) {
-    const int c = split * per_rank + threadIdx.x;
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
     float v = 0.f;
     if (live) {
-      for (int s = 0; s < S; ++s) {
-        float ms, as;
-        if constexpr (CLUSTER) {
-          ms = ld_peer_f32(peer_addr(my_f, s) + 4 * kSlotM);
-          as = ld_peer_f32(peer_addr(smem_addr(cta_acc + c), s));
-        } else {
-          ms = cta_f[kSlotM];
-          as = cta_acc[c];
-        }
-        if (ms != -INFINITY) v = fmaf(as, fast_exp2(ms - m_g), v);
+#pragma unroll
+      for (int w = 0; w < kNW; ++w) {
+        const float mw = table[split * kNW + w].x;
+        if (mw != -INFINITY) v = fmaf(fast_exp2(mw - m_g), wscr_of(w)[c], v);
       }
       v *= inv_z;
+      if (C::kLogits && gather) {
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) v += corr_of(w)[c];
+      }
     }
-    p.out[(static_cast<size_t>(b) * p.H + h) * D + c] = __float2bfloat16_rn(v);
+    const int slot = split * per_rank + c % per_rank;
+    if constexpr (CLUSTER) st_peer_f32(peer_addr(smem_addr(red + slot), c / per_rank), v);
+    else red[slot] = v;
+  }
+  if (threadIdx.x == 0) {
+    int total = 0;
+#pragma unroll
+    for (int w = 0; w < kNW; ++w) total += cta_i[kSlotCnt0 + w];
+    if constexpr (CLUSTER) st_peer_s32(peer_addr(smem_addr(cnts + split), 0), total);
+    else cnts[split] = total;
+  }
+  // after this barrier no CTA touches another's shared memory
+  if constexpr (CLUSTER) cluster_sync_all(); else __syncthreads();
+
+  if (threadIdx.x < per_rank) {
+    float v = 0.f;
+    for (int s = 0; s < S; ++s) v += red[s * per_rank + threadIdx.x];
+    p.out[(static_cast<size_t>(b) * p.H + h) * D + split * per_rank + threadIdx.x] = __float2bfloat16_rn(v);
   }
   if (split == 0 && threadIdx.x == 0) {
     if (p.sel_count) {
       int total = 0;
-      if (live && C::kQ4) {
-        for (int s = 0; s < S; ++s) {
-          if constexpr (CLUSTER) total += ld_peer_s32(peer_addr(smem_addr(&cta_i[kSlotCount]), s));
-          else total += cta_i[kSlotCount];
-        }
-      }
+      if (live && C::kQ4)
+        for (int s = 0; s < S; ++s) total += cnts[s];
       p.sel_count[static_cast<size_t>(b) * p.H + h] = total;
     }
     if (any_bad) flag_error(p.err, any_bad);
   }
-  if constexpr (CLUSTER) cluster_sync_all();  // peers' shared memory stays alive until here
 }
 
 template <int KIND, int D, bool FULLV, bool CLUSTER>
