@@ -157,7 +157,7 @@ struct Cfg {
   // same offsets of the two halves fall in different shared-memory banks
   static constexpr int kHalf = kLoad + 64;
   static constexpr int kStage = kHalf + kLoad;
-  static constexpr int kNSW = kQuant ? 3 : 2;              // ring stages per warp
+  static constexpr int kNSW = 2;                           // ring stages per warp
   static constexpr int kCH = 4;                            // lanes per token
   static constexpr int kCW = D / kCH;                      // channels per lane
   static constexpr int kNWRD = kCW / 16;                   // plane words per lane and token
@@ -276,26 +276,32 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
       alpha = a4;
     }
     __syncwarp();
-    float2 q2[CW / 2];
-#pragma unroll
-    for (int v = 0; v < CW / 4; ++v) {
-      const float4 x = *reinterpret_cast<const float4*>(q2buf + q2_slot<CW>(k, v));
-      q2[2 * v] = make_float2(x.x, x.y);
-      q2[2 * v + 1] = make_float2(x.z, x.w);
-    }
     // each of the CH lanes of a token starts from alpha / CH (exact: CH is a
     // power of two), so the all-reduce below adds alpha exactly once
     alpha *= pow2i(-C::kE) / CH;
+    float2 d[TPL];
 #pragma unroll
-    for (int j = 0; j < TPL; ++j) {
-      uint32_t hi[NWRD], lo[NWRD];
-      plane_words(j, R::kKHi, hi);
-      if constexpr (C::kQ4) plane_words(j, R::kQ4KLo, lo);
-      float2 d = make_float2(alpha, 0.f);
+    for (int j = 0; j < TPL; ++j) d[j] = make_float2(alpha, 0.f);
+    // one 16-channel word at a time: only its 8 coefficient pairs are live
 #pragma unroll
-      for (int u = 0; u < NWRD; ++u) d = dot16<C::kQ4>(q2 + 8 * u, hi[u], C::kQ4 ? lo[u] : 0u, d);
-      part[j] = d.x + d.y;
+    for (int u = 0; u < NWRD; ++u) {
+      float2 q2[8];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float4 x = *reinterpret_cast<const float4*>(q2buf + q2_slot<CW>(k, 4 * u + v));
+        q2[2 * v] = make_float2(x.x, x.y);
+        q2[2 * v + 1] = make_float2(x.z, x.w);
+      }
+#pragma unroll
+      for (int j = 0; j < TPL; ++j) {
+        uint32_t hi[NWRD], lo[NWRD] = {};
+        plane_words(j, R::kKHi, hi);
+        if constexpr (C::kQ4) plane_words(j, R::kQ4KLo, lo);
+        d[j] = dot16<C::kQ4>(q2, hi[u], lo[u], d[j]);
+      }
     }
+#pragma unroll
+    for (int j = 0; j < TPL; ++j) part[j] = d[j].x + d[j].y;
   } else if constexpr (C::kQuant) {
     // unfinished key group: exact bf16 keys from the residual
     const float* qf = qconst + CW * k;
@@ -416,11 +422,13 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
   }
 }
 
-template <int KIND, int D, bool FULLV, bool CLUSTER>
-__global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams p) {
+// MINB: CTAs per SM the register budget is cut for (4: 128 registers per
+// thread; 5: 102, for grids of many waves where occupancy pays).
+template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodeParams p) {
   using C = Cfg<KIND, D, FULLV>;
   using R = typename C::R;
-  constexpr int CH = C::kCH, CW = C::kCW, NWRD = C::kNWRD, TS = C::kTS, NSW = C::kNSW;
+  constexpr int CH = C::kCH, CW = C::kCW, NSW = C::kNSW;
   constexpr int LOAD = C::kLoad, STAGE = C::kStage;
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -799,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
   }
 }
 
-template <int KIND, int D, bool FULLV, bool CLUSTER>
+template <int KIND, int D, bool FULLV>
 size_t smem_bytes_t(int cg) {
   using C = Cfg<KIND, D, FULLV>;
   return smem_plan(C::kStage, C::kNSW, cg, D, C::kLogits).total;
@@ -807,11 +815,11 @@ size_t smem_bytes_t(int cg) {
 
 // CTAs of this instantiation that can be resident at once on the device
 // (for clusters: co-resident clusters times the cluster size).
-template <int KIND, int D, bool FULLV, bool CLUSTER>
+template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB>
 long resident_ctas_t(int cg, int splits, int sms) {
-  const size_t smem = smem_bytes_t<KIND, D, FULLV, CLUSTER>(cg);
+  const size_t smem = smem_bytes_t<KIND, D, FULLV>(cg);
   if (smem > 227u * 1024u) return 0;
-  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER>;
+  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return 0;
   if (!CLUSTER) {
@@ -835,11 +843,11 @@ long resident_ctas_t(int cg, int splits, int sms) {
   return static_cast<long>(clusters) * splits;
 }
 
-template <int KIND, int D, bool FULLV, bool CLUSTER>
+template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB>
 cudaError_t launch_t(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
-  const size_t smem = smem_bytes_t<KIND, D, FULLV, CLUSTER>(p.chunk_groups);
+  const size_t smem = smem_bytes_t<KIND, D, FULLV>(p.chunk_groups);
   if (smem > 227u * 1024u) return cudaErrorInvalidValue;
-  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER>;
+  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -866,27 +874,53 @@ cudaError_t launch_t(const DecodeParams& p, int batch, int splits, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
+template <int KIND, int D, bool FULLV, int MINB>
+long resident_m(int cg, int splits, int sms) {
+  return splits > 1 ? resident_ctas_t<KIND, D, FULLV, true, MINB>(cg, splits, sms)
+                    : resident_ctas_t<KIND, D, FULLV, false, MINB>(cg, splits, sms);
+}
+
+// A grid of at least this many waves of 4-per-SM residency runs the
+// 5-per-SM build: its extra warps hide latency once every SM stays busy for
+// long; short grids keep the full register budget.
+constexpr long kHighOccupancyWaves = 3;
+
 template <int KIND, int D, bool FULLV>
 cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
-  return splits > 1 ? launch_t<KIND, D, FULLV, true>(p, batch, splits, stream, pdl)
-                    : launch_t<KIND, D, FULLV, false>(p, batch, splits, stream, pdl);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  (void)sms;
+  if constexpr (KIND != LOOPKV_CELL_BF16 && !FULLV) {
+    const long ctas = static_cast<long>(batch) * p.H * splits;
+    const long slots4 = resident_m<KIND, D, FULLV, 4>(p.chunk_groups, splits, sms);
+    if (slots4 > 0 && ctas >= kHighOccupancyWaves * slots4 &&
+        resident_m<KIND, D, FULLV, 5>(p.chunk_groups, splits, sms) > slots4)
+      return splits > 1 ? launch_t<KIND, D, FULLV, true, 5>(p, batch, splits, stream, pdl)
+                        : launch_t<KIND, D, FULLV, false, 5>(p, batch, splits, stream, pdl);
+  }
+  return splits > 1 ? launch_t<KIND, D, FULLV, true, 4>(p, batch, splits, stream, pdl)
+                    : launch_t<KIND, D, FULLV, false, 4>(p, batch, splits, stream, pdl);
 }
 
-template <int KIND, int D, bool FULLV>
-long resident_c(int cg, int splits, int sms) {
-  return splits > 1 ? resident_ctas_t<KIND, D, FULLV, true>(cg, splits, sms)
-                    : resident_ctas_t<KIND, D, FULLV, false>(cg, splits, sms);
-}
-
-// Co-resident CTAs of one decode instantiation (0 without a device).
-long resident_ctas(int kind, int d, int cg, int splits, int sms) {
+// Co-resident CTAs of one decode build (0 without a device); minb 5 only
+// exists for the 4-bit and 2-bit kinds.
+long resident_ctas(int kind, int d, int cg, int splits, int sms, int minb) {
+  if (minb == 5) {
+    switch (kind * 1000 + d) {
+      case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 5>(cg, splits, sms);
+      case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 5>(cg, splits, sms);
+      case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 5>(cg, splits, sms);
+      case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 5>(cg, splits, sms);
+      default: return 0;
+    }
+  }
   switch (kind * 1000 + d) {
-    case LOOPKV_CELL_Q4 * 1000 + 128: return resident_c<LOOPKV_CELL_Q4, 128, false>(cg, splits, sms);
-    case LOOPKV_CELL_Q4 * 1000 + 64: return resident_c<LOOPKV_CELL_Q4, 64, false>(cg, splits, sms);
-    case LOOPKV_CELL_Q2 * 1000 + 128: return resident_c<LOOPKV_CELL_Q2, 128, false>(cg, splits, sms);
-    case LOOPKV_CELL_Q2 * 1000 + 64: return resident_c<LOOPKV_CELL_Q2, 64, false>(cg, splits, sms);
-    case LOOPKV_CELL_BF16 * 1000 + 128: return resident_c<LOOPKV_CELL_BF16, 128, false>(cg, splits, sms);
-    case LOOPKV_CELL_BF16 * 1000 + 64: return resident_c<LOOPKV_CELL_BF16, 64, false>(cg, splits, sms);
+    case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 4>(cg, splits, sms);
+    case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 4>(cg, splits, sms);
+    case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 4>(cg, splits, sms);
+    case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 4>(cg, splits, sms);
+    case LOOPKV_CELL_BF16 * 1000 + 128: return resident_m<LOOPKV_CELL_BF16, 128, false, 4>(cg, splits, sms);
+    case LOOPKV_CELL_BF16 * 1000 + 64: return resident_m<LOOPKV_CELL_BF16, 64, false, 4>(cg, splits, sms);
     default: return 0;
   }
 }
@@ -904,18 +938,28 @@ int decode_splits(int kind, int head_dim, int batch, int heads, int max_seq_len)
   if (pairs <= 0 || groups <= 1) return min_s;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Score of a split count: for a short grid, the fraction of the resident
+  // slots its waves keep busy; for a long grid (the launch then runs the
+  // 5-per-SM build where that fits more CTAs), busy slots per SM relative to
+  // four, so that more resident warps win once every SM stays loaded.
   int best = min_s;
-  double best_eff = -1.0;
+  double best_score = -1.0;
   for (int s = min_s; s <= 8; s <<= 1) {
     if (s > min_s && groups < 2 * kNW * s) break;  // keep >= 2 groups per warp
     const int cg = (groups + s - 1) / s;
-    long slots = resident_ctas(kind, head_dim, cg, s, sms);
+    long slots = resident_ctas(kind, head_dim, cg, s, sms, 4);
     if (slots <= 0) slots = 4L * sms;  // no device: a fixed guess keeps the choice deterministic
     const long ctas = pairs * s;
+    const bool long_grid = ctas >= kHighOccupancyWaves * slots;
+    if (long_grid) {
+      const long slots5 = resident_ctas(kind, head_dim, cg, s, sms, 5);
+      if (slots5 > slots) slots = slots5;
+    }
     const long waves = (ctas + slots - 1) / slots;
     const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
-    if (eff > best_eff + 0.02) {
-      best_eff = eff;
+    const double score = long_grid ? eff * static_cast<double>(slots) / (4.0 * sms) : eff;
+    if (score > best_score + 0.02) {
+      best_score = score;
       best = s;
     }
   }
