@@ -33,6 +33,7 @@
 // (values).  Subnormal FMA inputs are exact on this hardware (no FTZ), so
 // every product equals q * scale * code up to the global power of two 2^-E.
 #include <float.h>
+#include <limits.h>
 
 #include <algorithm>
 
@@ -146,6 +147,38 @@ __device__ __forceinline__ void axpy16_h(float2* acc, uint32_t wh, uint32_t x) {
   }
 }
 
+// Index of the sequence with rank r when the batch is ordered by decreasing
+// length, ties by increasing index (a bijection of [0, B)).  Batches of
+// equal lengths, or of more than kMaxRankedBatch sequences, keep the
+// identity.  Every lane of the warp must call it; lengths are compared as
+// given (a bad length only moves that sequence in the order).
+constexpr int kMaxRankedBatch = 64;
+__device__ __forceinline__ int sequence_of_rank(const int32_t* seq_lens, int B, int r, int lane) {
+  if (B > kMaxRankedBatch) return r;
+  const int n0 = lane < B ? seq_lens[lane] : 0;
+  const int n1 = lane + 32 < B ? seq_lens[lane + 32] : 0;
+  const int mn = __reduce_min_sync(0xffffffffu, lane < B ? (lane + 32 < B ? min(n0, n1) : n0) : INT_MAX);
+  const int mx = __reduce_max_sync(0xffffffffu, lane < B ? (lane + 32 < B ? max(n0, n1) : n0) : INT_MIN);
+  if (mn == mx) return r;
+  int found = -1;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int bb = lane + 32 * half;
+    const int nb = half ? n1 : n0;
+    int rank = 0;
+    for (int i = 0; i < min(B, 32); ++i) {
+      const int n2 = __shfl_sync(0xffffffffu, n0, i);
+      rank += (n2 > nb) || (n2 == nb && i < bb);
+    }
+    for (int i = 32; i < B; ++i) {
+      const int n2 = __shfl_sync(0xffffffffu, n1, i - 32);
+      rank += (n2 > nb) || (n2 == nb && i < bb);
+    }
+    if (bb < B && rank == r) found = bb;
+  }
+  return __reduce_max_sync(0xffffffffu, found);
+}
+
 template <int KIND, int D, bool FULLV>
 struct Cfg {
   using R = Rec<KIND, D>;
@@ -175,9 +208,9 @@ struct Cfg {
 };
 
 // Shared-memory carve-up (bytes), identical on host and device.
-// After pass 1 a warp's ring is idle and holds the warp's results: its
-// per-channel sums (wscr, at the ring's start) and its low-plane corrections
-// (at +kCorrOff).  The exchange area (xchg) is never aliased: peers of the
+// After pass 1 a warp's ring is idle and holds the warp's results: the
+// per-channel partial sums of its TS token sub-groups (wscr, at the ring's
+// start) and its low-plane corrections (after them).  The exchange area (xchg) is never aliased: peers of the
 // cluster store into it while this CTA may still be in pass 1.
 //   xchg: table float4[8 * kNW] (every warp's max, sum, error bits),
 //         red float[D] (the owner's slice sums of every split),
@@ -185,7 +218,6 @@ struct Cfg {
 struct Smem {
   size_t rings, ring_bytes, bars, qconst, q2buf, logits, ids, masks, xchg, scal, total;
 };
-constexpr int kCorrOff = 1024;
 __host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int d, bool logits) {
   Smem s;
   s.rings = 0;
@@ -205,6 +237,14 @@ __host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int 
 
 // Per-CTA scalar slots.
 enum { kSlotBad = 0, kSlotCnt0 = 4 };
+
+// 16-byte piece (of CW / 4) where lane (r, k) stores channels 4v .. 4v + 3
+// of its chunk: the rotation by 2k + r puts the eight lanes of each store
+// phase on distinct bank groups (CW = 32).
+template <int CW>
+__host__ __device__ __forceinline__ int wscr_piece(int v, int k, int r) {
+  return (v + 2 * k + r) & (CW / 4 - 1);
+}
 
 // Per-lane running state of one warp's online softmax.
 template <int CW>
@@ -428,13 +468,14 @@ template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB>
 __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodeParams p) {
   using C = Cfg<KIND, D, FULLV>;
   using R = typename C::R;
-  constexpr int CH = C::kCH, CW = C::kCW, NSW = C::kNSW;
+  constexpr int CH = C::kCH, CW = C::kCW, NSW = C::kNSW, TS = C::kTS;
   constexpr int LOAD = C::kLoad, STAGE = C::kStage;
 
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem sp = smem_plan(STAGE, NSW, p.chunk_groups, D, C::kLogits);
   float* logits = reinterpret_cast<float*>(smem + sp.logits);
   auto wscr_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w); };
+  constexpr int kCorrOff = TS * D * 4;  // after the warp's TS x D partial sums
   auto corr_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w + kCorrOff); };
   int32_t* ids_smem = reinterpret_cast<int32_t*>(smem + sp.ids);
   uint32_t* masks_smem = reinterpret_cast<uint32_t*>(smem + sp.masks);
@@ -442,12 +483,16 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   float* red = reinterpret_cast<float*>(smem + sp.xchg + 16 * 8 * kNW);
   int* cnts = reinterpret_cast<int*>(smem + sp.xchg + 16 * 8 * kNW + 4 * D);
   int* cta_i = reinterpret_cast<int*>(smem + sp.scal);
-  static_assert(D * 4 <= kCorrOff && kCorrOff + D * 4 <= NSW * STAGE, "warp results must fit in an idle ring");
+  static_assert(kCorrOff + D * 4 <= NSW * STAGE, "warp results must fit in an idle ring");
 
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, h = blockIdx.y;
   const int S = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_allow_dependents();
+  // Clusters are dispatched roughly in launch order; the z-th batch slot
+  // takes the sequence of rank z by decreasing length (ties by index), so
+  // ragged batches start their longest sequences first.
+  const int b = sequence_of_rank(p.seq_lens, static_cast<int>(gridDim.z), static_cast<int>(blockIdx.z), lane);
 
   // ---- this split's chunk of 32-token groups (seq_lens and the block table
   //      are not written by the previous kernel: read before its completion)
@@ -607,16 +652,14 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     }
     lw = ws.l * unsh;
 #pragma unroll
-    for (int off = CH; off < 32; off <<= 1) {
+    for (int off = CH; off < 32; off <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+    // every lane stores its partial sums; the combine adds the TS token
+    // sub-groups (16-byte pieces rotated so that each store is conflict-free)
+    float* wsc = wscr_of(warp) + r * D + k * CW;
 #pragma unroll
-      for (int i = 0; i < CW; ++i) o[i] += __shfl_xor_sync(0xffffffffu, o[i], off);
-      lw += __shfl_xor_sync(0xffffffffu, lw, off);
-    }
-    float* wsc = wscr_of(warp);
-    if (r == 0) {
-#pragma unroll
-      for (int i = 0; i < CW; ++i) wsc[CW * k + i] = o[i];
-    }
+    for (int v = 0; v < CW / 4; ++v)
+      *reinterpret_cast<float4*>(wsc + 4 * wscr_piece<CW>(v, k, r)) =
+          make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
   }
 
   // ---- publish (max, sum, error bits) of this warp into every split's table
@@ -766,10 +809,17 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     const int c = threadIdx.x;
     float v = 0.f;
     if (live) {
+      const int kc = c / CW, i = c % CW;
 #pragma unroll
       for (int w = 0; w < kNW; ++w) {
         const float mw = table[split * kNW + w].x;
-        if (mw != -INFINITY) v = fmaf(fast_exp2(mw - m_g), wscr_of(w)[c], v);
+        if (mw != -INFINITY) {
+          const float* wsc = wscr_of(w) + kc * CW + (i & 3);
+          float sw = 0.f;
+#pragma unroll
+          for (int rr = 0; rr < TS; ++rr) sw += wsc[rr * D + 4 * wscr_piece<CW>(i >> 2, kc, rr)];
+          v = fmaf(fast_exp2(mw - m_g), sw, v);
+        }
       }
       v *= inv_z;
       if (C::kLogits && gather) {
