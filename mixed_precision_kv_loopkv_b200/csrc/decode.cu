@@ -68,9 +68,15 @@ __device__ __forceinline__ float nib(uint32_t w, uint32_t w20, int m) {
 }
 // Full 4-bit codes of 16 channels from their high and low plane words:
 // even = channels 0,2,..,14 in nibbles 0..7; odd = channels 1,3,..,15.
+// (a & c) | (b & ~c) in one LOP3
+__device__ __forceinline__ uint32_t bit_select(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 __device__ __forceinline__ void combine_planes(uint32_t hi, uint32_t lo, uint32_t& even, uint32_t& odd) {
-  even = ((hi << 2) & 0xCCCCCCCCu) | (lo & 0x33333333u);
-  odd = (hi & 0xCCCCCCCCu) | ((lo >> 2) & 0x33333333u);
+  even = bit_select(hi << 2, lo, 0xCCCCCCCCu);
+  odd = bit_select(hi, lo >> 2, 0xCCCCCCCCu);
 }
 
 // Dot product of the subnormal code views of one 16-channel word with 8
@@ -608,6 +614,9 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       const int stage = it % NSW;
       if (!mbar_wait(bar0 + 8 * stage, (it / NSW) & 1)) {
         atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_TIMEOUT);
+        // give the copies still in flight one more bounded wait before this
+        // CTA moves on (and eventually releases its shared memory)
+        for (int pend = it; pend < min(nit, it + NSW); ++pend) mbar_wait(bar0 + 8 * (pend % NSW), (pend / NSW) & 1);
         break;
       }
       const int gi = warp + kNW * it;
