@@ -97,8 +97,9 @@ typedef enum {
 /* loopkv_config.flags */
 #define LOOPKV_FLAG_PDL 0x1 /* programmatic dependent launch: a kernel may start
                                while the previous kernel on the stream drains.
-                               The append kernel waits for it before touching
-                               memory.  The decode kernel reads seq_lens and the
+                               The append kernel reads start_pos and the block
+                               table before it waits, and touches nothing else
+                               until then.  The decode kernel reads seq_lens and the
                                block table, and streams the cache blocks of the
                                32-token groups before the one holding token
                                seq_len - 1, before it waits: the previous kernel

@@ -82,18 +82,22 @@ template <int KIND, int D>
 __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
   using R = Rec<KIND, D>;
   // Let the next kernel (a decode of this cell) launch and stream the cache
-  // blocks this kernel does not write; then wait for the kernel before this
-  // one, which may produce the new tokens.
+  // blocks this kernel does not write.
   pdl_allow_dependents();
-  pdl_wait_prior_grid();
 
   const int h = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.T;
+  // The start position and the block table are not written by the previous
+  // kernel: read them (and the first new token's record) before waiting.
   const int start = p.start_pos[b];
   const int end = start + T;
+  const bool in_range = start >= 0 && end <= p.max_blocks * kBlock;
+  uint8_t* const rec_first = in_range ? record_of<KIND, D>(p, b, h, start) : nullptr;
+  // then wait for the kernel before this one, which may produce the new tokens
+  pdl_wait_prior_grid();
   if (start < 0) return;  // sequence not appended to in this call
-  if (end > p.max_blocks * kBlock) {
+  if (!in_range) {
     if (threadIdx.x == 0) flag_error(p.err, LOOPKV_DEVERR_SEQ_LEN);
     return;
   }
@@ -106,7 +110,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
     for (int i = threadIdx.x; i < T * kVecPerRow; i += blockDim.x) {
       const int t = i / kVecPerRow, c = i % kVecPerRow;
       const int pos = start + t;
-      uint8_t* rec = record_of<KIND, D>(p, b, h, pos);
+      uint8_t* rec = t == 0 ? rec_first : record_of<KIND, D>(p, b, h, pos);
       if (!rec) continue;
       const int row = pos % kBlock;
       reinterpret_cast<uint4*>(rec + R::kBfK + row * D * 2)[c] =
@@ -131,7 +135,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
       const uint32_t shift = 2u * (lane & 15);
       const uint32_t w_hi = half_warp_or((kSplit ? code >> 2 : code) << shift);
       const uint32_t w_lo = kSplit ? half_warp_or((code & 3u) << shift) : 0u;
-      uint8_t* rec = record_of<KIND, D>(p, b, h, pos);
+      uint8_t* rec = t == 0 ? rec_first : record_of<KIND, D>(p, b, h, pos);
       if (!rec) continue;
       const int row = pos % kBlock;
       if ((lane & 15) == 0) {
