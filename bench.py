@@ -5,9 +5,10 @@ Metric: decode-attention KV GB/s (algorithmic bytes the decode kernels must
 move, over device time) and microseconds per looped decode step.
 
 One step = every (loop, layer) cell of the Ouro-1.4B-like workload in order:
-stored cells append the current token (quantise-append kernel) and attend
-over n + 1 tokens, reuse cells attend over the final loop's n tokens (fused
-decode-attention kernel).  The step is captured once in a CUDA graph (kernels
+stored cells append the current token and attend over n + 1 tokens in one
+launch (loopkv_append_decode_attention; --no-fuse: append kernel, then decode
+kernel), reuse cells attend over the final loop's n tokens
+(loopkv_decode_attention).  The step is captured once in a CUDA graph (kernels
 launched with programmatic dependent launch) and replayed.  Every step
 decodes at the same position (the append rewrites the same token), so the
 context stays at the workload's length however many steps are timed.
@@ -50,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="ouro_step")
     ap.add_argument("--splits", type=int, default=0, help="decode splits override (0 = automatic)")
     ap.add_argument("--no-pdl", action="store_true")
+    ap.add_argument("--no-fuse", action="store_true",
+                    help="stored cells append and attend in two launches instead of one")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
@@ -196,7 +199,7 @@ def profiled_traffic(workload: str):
 
 # ----------------------------------------------------------------- workload setup
 
-def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0):
+def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0, fused: bool = True):
     from mixed_precision_kv_loopkv_b200 import LOOPKV_FLAG_PDL, KVCells, LoopedDecodeStep, prefill
     from workload import block_table_for, cell_kv, cell_new_token, cell_query, make_plan, seq_lens_for
 
@@ -235,7 +238,7 @@ def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0):
         kv, table, pos, [q_all[c] for c in range(C)],
         {c: kn_all[slot[c]] for c in stored}, {c: vn_all[slot[c]] for c in stored},
         [out_all[c] for c in range(C)], w.tau, w.sm_scale, int(lens.max()) + 1,
-        sel_count=[sel_all[c] for c in range(C)], cells=run)
+        sel_count=[sel_all[c] for c in range(C)], cells=run, fused=fused)
     torch.cuda.synchronize()
     return dict(plan=plan, lens=lens, kv=kv, step=step, q_all=q_all, kn_all=kn_all, vn_all=vn_all,
                 out_all=out_all, sel_all=sel_all)
@@ -382,7 +385,7 @@ def main_arm(args, world, rank, local):
     w = get_workload(args.workload)
     if args.batch:
         w = w.with_(batch=args.batch)
-    S = setup(w, pdl=not args.no_pdl, splits=args.splits, ncells=args.cells)
+    S = setup(w, pdl=not args.no_pdl, splits=args.splits, ncells=args.cells, fused=not args.no_fuse)
     step, plan, lens = S["step"], S["plan"], S["lens"]
     dev = torch.device(f"cuda:{local}")
 
@@ -448,7 +451,8 @@ def main_arm(args, world, rank, local):
         cfg = workload_config(w, world)
         if args.cells:
             cfg["cells_run"] = len(step.cells)
-        cfg.update({"pdl": not args.no_pdl, "splits": args.splits or "auto", "cuda_graph": True,
+        cfg.update({"pdl": not args.no_pdl, "fused_append": not args.no_fuse,
+                    "splits": args.splits or "auto", "cuda_graph": True,
                     "algorithmic_bytes_per_step": bytes_step,
                     "selected_low_plane_rows_per_step": int(sel.sum())})
         line = {

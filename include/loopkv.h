@@ -189,6 +189,30 @@ LOOPKV_API loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const
                                       float sm_scale, void* out, uint32_t* sel_mask,
                                       int32_t* sel_count, int32_t* err_flag, void* stream);
 
+/*
+ * One decode step of a stored cell in a single launch: appends token
+ * start_pos[b] (one new token per sequence) exactly as loopkv_quantize_append
+ * with num_tokens = 1 would, then attends over start_pos[b] + 1 tokens exactly
+ * as loopkv_decode_attention would with seq_lens = start_pos + 1.  This is
+ * the single fused kernel per cell the LoopKV abstract describes, with the
+ * store of the current token folded into it: the split holding the new
+ * token writes it before it reads that token's group.
+ *
+ *   k_new, v_new : device bf16 [batch][1][H][D]
+ *   start_pos    : device int32 [batch]; a negative entry skips that sequence
+ *                  (nothing stored, zeros out)
+ *   max_seq_len  : host upper bound on start_pos + 1; 0 means the capacity
+ *   other arguments as for loopkv_decode_attention
+ * Errors: as loopkv_decode_attention, and INVALID_ARG for a reuse cell or
+ * null k_new / v_new.  Device faults: LOOPKV_DEVERR_SEQ_LEN for start_pos + 1
+ * above max_seq_len or the capacity, BLOCK_ID, RANGE as for the append.
+ */
+LOOPKV_API loopkv_status loopkv_append_decode_attention(
+    const loopkv_config* cfg, const loopkv_cells* cells, int32_t loop, int32_t layer, const void* k_new,
+    const void* v_new, const void* q, const int32_t* block_table, const int32_t* start_pos, int32_t batch,
+    int32_t max_seq_len, float tau, float sm_scale, void* out, uint32_t* sel_mask, int32_t* sel_count,
+    int32_t* err_flag, void* stream);
+
 /* Context splits (CTAs per sequence and head) a decode call over a source
  * cell of the given kind would launch; 0 for invalid arguments. */
 LOOPKV_API int32_t loopkv_decode_splits(const loopkv_config* cfg, int32_t kind, int32_t batch,

@@ -23,6 +23,7 @@ from .loopkv import (  # noqa: F401
     KVCells,
     LoopKVError,
     library,
+    loopkv_append_decode_attention,
     loopkv_decode_attention,
     loopkv_decode_splits,
     loopkv_quantize_append,

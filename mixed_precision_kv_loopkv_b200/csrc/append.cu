@@ -16,67 +16,11 @@
 //      exact ones waiting in the key residual; planes and meta written;
 //   3. after a CTA barrier, the new tokens of the still-open group are copied
 //      into the key residual (after step 2 read the residual).
-#include "device_common.cuh"
+#include "append_ops.cuh"
 #include "kernels.h"
 
 namespace loopkv {
 namespace {
-
-// Largest value-group scale the decode kernel's f16 value weights carry.
-constexpr float kMaxValueScale = 255.f;
-
-__device__ __forceinline__ float warp_min(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
-}
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
-}
-// OR over the 16 lanes of each half-warp.
-__device__ __forceinline__ uint32_t half_warp_or(uint32_t x) {
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) x |= __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
-}
-
-// bf16 scale and minimum of a group with extremes mn, mx.
-template <int BITS>
-__device__ __forceinline__ void group_params(float mn, float mx, float& s_b, float& mn_b) {
-  mn_b = __bfloat162float(__float2bfloat16_rn(mn));
-  const float s = __fdiv_rn(__fsub_rn(mx, mn_b), static_cast<float>((1 << BITS) - 1));
-  s_b = __bfloat162float(__float2bfloat16_rn(s));
-}
-
-template <int BITS>
-__device__ __forceinline__ uint32_t group_code(float x, float s_b, float mn_b) {
-  if (s_b == 0.f) return 0u;
-  float t = rintf(__fdiv_rn(__fsub_rn(x, mn_b), s_b));
-  t = fminf(fmaxf(t, 0.f), static_cast<float>((1 << BITS) - 1));
-  return static_cast<uint32_t>(t);
-}
-
-__device__ __forceinline__ uint32_t meta_word(float s_b, float mn_b) {
-  return static_cast<uint32_t>(bf16_bits_rn(s_b)) |
-         (static_cast<uint32_t>(bf16_bits_rn(mn_b)) << 16);
-}
-
-template <int KIND, int D>
-__device__ __forceinline__ uint8_t* record_of(const AppendParams& p, int b, int h, int pos) {
-  const int lb = pos / kBlock;
-  if (lb >= p.max_blocks) {
-    flag_error(p.err, LOOPKV_DEVERR_SEQ_LEN);
-    return nullptr;
-  }
-  const int phys = p.block_table[static_cast<size_t>(b) * p.max_blocks + lb];
-  if (phys < 0 || phys >= p.num_blocks) {
-    flag_error(p.err, LOOPKV_DEVERR_BLOCK_ID);
-    return nullptr;
-  }
-  return p.arena + (static_cast<size_t>(phys) * p.H + h) * Rec<KIND, D>::kBytes;
-}
 
 template <int KIND, int D>
 __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
@@ -93,7 +37,9 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
   const int start = p.start_pos[b];
   const int end = start + T;
   const bool in_range = start >= 0 && end <= p.max_blocks * kBlock;
-  uint8_t* const rec_first = in_range ? record_of<KIND, D>(p, b, h, start) : nullptr;
+  const CellRows cell{p.arena, p.block_table + static_cast<size_t>(b) * p.max_blocks, p.err, p.H, h,
+                      p.max_blocks, p.num_blocks};
+  uint8_t* const rec_first = in_range ? record_at<KIND, D>(cell, start) : nullptr;
   // then wait for the kernel before this one, which may produce the new tokens
   pdl_wait_prior_grid();
   if (start < 0) return;  // sequence not appended to in this call
@@ -110,7 +56,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
     for (int i = threadIdx.x; i < T * kVecPerRow; i += blockDim.x) {
       const int t = i / kVecPerRow, c = i % kVecPerRow;
       const int pos = start + t;
-      uint8_t* rec = t == 0 ? rec_first : record_of<KIND, D>(p, b, h, pos);
+      uint8_t* rec = t == 0 ? rec_first : record_at<KIND, D>(cell, pos);
       if (!rec) continue;
       const int row = pos % kBlock;
       reinterpret_cast<uint4*>(rec + R::kBfK + row * D * 2)[c] =
@@ -120,8 +66,6 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
     }
     return;
   } else {
-    constexpr int BITS = KIND == LOOPKV_CELL_Q4 ? 4 : 2;
-    constexpr bool kSplit = KIND == LOOPKV_CELL_Q4;
     constexpr int kVGroups = D / kGroup;
 
     // 1. values, one token and 32-channel group per warp iteration
@@ -129,63 +73,18 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
       const int t = item / kVGroups, g = item % kVGroups;
       const int pos = start + t;
       const float x = __bfloat162float(vb[t * tok_stride + g * kGroup + lane]);
-      float s_b, mn_b;
-      group_params<BITS>(warp_min(x), warp_max(x), s_b, mn_b);
-      const uint32_t code = group_code<BITS>(x, s_b, mn_b);
-      const uint32_t shift = 2u * (lane & 15);
-      const uint32_t w_hi = half_warp_or((kSplit ? code >> 2 : code) << shift);
-      const uint32_t w_lo = kSplit ? half_warp_or((code & 3u) << shift) : 0u;
-      uint8_t* rec = t == 0 ? rec_first : record_of<KIND, D>(p, b, h, pos);
-      if (!rec) continue;
-      const int row = pos % kBlock;
-      if ((lane & 15) == 0) {
-        const int word = 2 * g + (lane >> 4);
-        *reinterpret_cast<uint32_t*>(rec + R::kVHi + row * R::kRow + word * 4) = w_hi;
-        if constexpr (kSplit)
-          *reinterpret_cast<uint32_t*>(rec + R::kQ4VLo + row * R::kRow + word * 4) = w_lo;
-      }
-      if (lane == 0) {
-        *reinterpret_cast<uint32_t*>(rec + R::kVMetaOff + (row * kVGroups + g) * 4) =
-            meta_word(s_b, mn_b);
-        if (s_b > kMaxValueScale) flag_error(p.err, LOOPKV_DEVERR_RANGE);
-      }
+      uint8_t* rec = t == 0 ? rec_first : record_at<KIND, D>(cell, pos);
+      store_value_group<KIND, D>(rec, pos % kBlock, g, x, lane, p.err);
     }
 
     // 2. key groups completed by this call: groups [start/32, end/32 - 1]
     __nv_bfloat16* res = p.residual + (static_cast<size_t>(b) * p.H + h) * kGroup * D;
     const int g_first = start / kGroup, g_last = end / kGroup - 1;
-    constexpr int kChunks = D / 16;
     for (int G = g_first; G <= g_last; ++G) {
       const int pos = G * kGroup + lane;  // this lane's token
       const __nv_bfloat16* src =
           pos >= start ? kb + static_cast<size_t>(pos - start) * tok_stride : res + lane * D;
-      for (int ck = warp; ck < kChunks; ck += 4) {
-        uint32_t w_hi = 0, w_lo = 0;
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-          const int c = ck * 16 + i;
-          const float x = __bfloat162float(src[c]);
-          float s_b, mn_b;
-          group_params<BITS>(warp_min(x), warp_max(x), s_b, mn_b);
-          const uint32_t code = group_code<BITS>(x, s_b, mn_b);
-          w_hi |= (kSplit ? code >> 2 : code) << (2 * i);
-          if constexpr (kSplit) w_lo |= (code & 3u) << (2 * i);
-          if (lane == 0) {
-            // channels [0, D/2) live in the group's even block, the rest in the odd one
-            uint8_t* mrec = record_of<KIND, D>(p, b, h, G * kGroup + (c < D / 2 ? 0 : kBlock));
-            if (mrec)
-              *reinterpret_cast<uint32_t*>(mrec + R::kKMetaOff + (c % (D / 2)) * 4) =
-                  meta_word(s_b, mn_b);
-          }
-        }
-        uint8_t* rec = record_of<KIND, D>(p, b, h, pos);
-        if (rec) {
-          const int row = pos % kBlock;
-          *reinterpret_cast<uint32_t*>(rec + R::kKHi + row * R::kRow + ck * 4) = w_hi;
-          if constexpr (kSplit)
-            *reinterpret_cast<uint32_t*>(rec + R::kQ4KLo + row * R::kRow + ck * 4) = w_lo;
-        }
-      }
+      store_key_group<KIND, D>(cell, G, src, warp, lane, 4);
     }
     __syncthreads();
 

@@ -39,6 +39,7 @@
 
 #include <cuda_fp16.h>
 
+#include "append_ops.cuh"
 #include "device_common.cuh"
 #include "kernels.h"
 
@@ -183,6 +184,39 @@ __device__ __forceinline__ int sequence_of_rank(const int32_t* seq_lens, int B, 
     if (bb < B && rank == r) found = bb;
   }
   return __reduce_max_sync(0xffffffffu, found);
+}
+
+// The decode step's append of one token at position pos into (b, h), run by
+// every thread of the CTA that holds the token's group: the value row (both
+// planes and meta) from v_new; the key either joins the exact residual or,
+// as its group's 32nd token, completes the group, which is then quantised
+// per channel from the residual.
+template <int KIND, int D>
+__device__ __forceinline__ void append_token(const DecodeParams& p, int b, int h, int pos, int warp, int lane) {
+  using R = Rec<KIND, D>;
+  const CellRows cell{p.wr_arena, p.block_table + static_cast<size_t>(b) * p.max_blocks, p.err, p.H, h,
+                      p.max_blocks, p.num_blocks};
+  const __nv_bfloat16* kb = p.k_new + (static_cast<size_t>(b) * p.H + h) * D;
+  const __nv_bfloat16* vb = p.v_new + (static_cast<size_t>(b) * p.H + h) * D;
+  uint8_t* rec = record_at<KIND, D>(cell, pos);
+  const int row = pos % kBlock;
+  if constexpr (KIND == LOOPKV_CELL_BF16) {
+    constexpr int kVec = D * 2 / 16;
+    if (rec && static_cast<int>(threadIdx.x) < 2 * kVec) {
+      const int c = threadIdx.x % kVec;
+      const bool value = static_cast<int>(threadIdx.x) >= kVec;
+      reinterpret_cast<uint4*>(rec + (value ? R::kBfV : R::kBfK) + row * D * 2)[c] =
+          reinterpret_cast<const uint4*>(value ? vb : kb)[c];
+    }
+  } else {
+    if (warp < D / kGroup) store_value_group<KIND, D>(rec, row, warp, __bfloat162float(vb[warp * kGroup + lane]), lane, p.err);
+    __nv_bfloat16* res = p.wr_residual + (static_cast<size_t>(b) * p.H + h) * kGroup * D;
+    if (pos % kGroup == kGroup - 1) {
+      store_key_group<KIND, D>(cell, pos / kGroup, lane == kGroup - 1 ? kb : res + lane * D, warp, lane, kNW);
+    } else if (static_cast<int>(threadIdx.x) < D * 2 / 16) {
+      reinterpret_cast<uint4*>(res + (pos % kGroup) * D)[threadIdx.x] = reinterpret_cast<const uint4*>(kb)[threadIdx.x];
+    }
+  }
 }
 
 template <int KIND, int D, bool FULLV>
@@ -456,6 +490,9 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
       const uint4* vp = reinterpret_cast<const uint4*>(st + ((TS * j) >> 4) * HALF + R::kBfV +
                                                        (r + ((TS * j) & 15)) * D * 2 + 2 * CW * k);
       const float2 ww = make_float2(wgt[j], wgt[j]);
+      // past the end of the tail group the stage holds stale bytes, which
+      // may read as Inf / NaN: skip them rather than multiply by zero
+      if (TAIL && tok0 + r + TS * j >= nn) continue;
 #pragma unroll
       for (int v = 0; v < CW / 8; ++v) {
         const uint4 a = vp[v];
@@ -502,7 +539,8 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
 
   // ---- this split's chunk of 32-token groups (seq_lens and the block table
   //      are not written by the previous kernel: read before its completion)
-  const int n = p.seq_lens[b];
+  const bool fused_append = p.k_new != nullptr;
+  const int n = fused_append ? (p.seq_lens[b] >= 0 ? p.seq_lens[b] + 1 : 0) : p.seq_lens[b];
   int bad = 0;
   if (n < 0 || n > p.max_seq_len || n > p.max_blocks * kBlock) bad = LOOPKV_DEVERR_SEQ_LEN;
   const int nn = bad ? 0 : n;
@@ -584,10 +622,20 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   };
 
   // ---- pass 1
-  if (nit > 0) {
-    int issued = 0;
+  int issued = 0;
+  if (nit > 0)
     while (issued < NSW && issued < nit && g0 + warp + kNW * issued < g_unsafe) issue(issued++);
-    pdl_wait_prior_grid();  // q, the residual and the newest group may come from the previous kernel
+  pdl_wait_prior_grid();  // q, the residual and the newest group may come from the previous kernel
+  if (fused_append) {
+    // the split holding the new token stores it first; its copies of the
+    // newest group are issued after the writes are visible to the bulk copies
+    if (!bad && nn > 0 && (nn - 1) / kGroup >= g0 && (nn - 1) / kGroup < g0 + cg) {
+      append_token<KIND, D>(p, b, h, nn - 1, warp, lane);
+      fence_proxy_async_global();
+    }
+    __syncthreads();
+  }
+  if (nit > 0) {
     while (issued < NSW) issue(issued++);
 
     // query constants (log2 units): qf_c, and qs_c = qf_c * 2^(149 - pos - E)

@@ -34,6 +34,13 @@ struct DecodeParams {
   int max_seq_len;
   float tau;
   float sm_scale_log2;            // sm_scale * log2(e)
+  // fused append (k_new non-null): seq_lens holds start positions; the
+  // kernel first stores token start_pos[b] into the cell, then attends over
+  // start_pos[b] + 1 tokens (negative start: sequence skipped)
+  const __nv_bfloat16* k_new;     // [B][1][H][D]
+  const __nv_bfloat16* v_new;     // [B][1][H][D]
+  uint8_t* wr_arena;              // the same arena, writable
+  __nv_bfloat16* wr_residual;     // the same key residual, writable
 };
 
 cudaError_t launch_append(int kind, int head_dim, const AppendParams& p, int batch,

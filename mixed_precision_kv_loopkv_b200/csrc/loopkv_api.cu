@@ -119,17 +119,25 @@ int32_t loopkv_decode_splits(const loopkv_config* cfg, int32_t kind, int32_t bat
   return loopkv::decode_splits(kind, cfg->head_dim, batch, cfg->num_heads, len);
 }
 
-loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const loopkv_cells* cells,
-                                      int32_t loop, int32_t layer, const void* q,
-                                      const int32_t* block_table, const int32_t* seq_lens,
-                                      int32_t batch, int32_t max_seq_len, float tau,
-                                      float sm_scale, void* out, uint32_t* sel_mask,
-                                      int32_t* sel_count, int32_t* err_flag, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared by the plain decode and the fused append + decode: validation,
+// split choice and launch.  k_new == nullptr: plain decode over seq_lens;
+// otherwise seq_lens holds start positions and the cell must be stored.
+loopkv_status decode_common(const loopkv_config* cfg, const loopkv_cells* cells, int32_t loop, int32_t layer,
+                            const void* k_new, const void* v_new, const void* q, const int32_t* block_table,
+                            const int32_t* seq_lens, int32_t batch, int32_t max_seq_len, float tau,
+                            float sm_scale, void* out, uint32_t* sel_mask, int32_t* sel_count,
+                            int32_t* err_flag, void* stream) {
   loopkv_status st = check_config(cfg);
   if (st != LOOPKV_OK) return st;
   int cell;
   if ((st = cell_index(cfg, loop, layer, &cell)) != LOOPKV_OK) return st;
+  const bool fused = k_new != nullptr || v_new != nullptr;
   // a reuse cell reads the final loop's cell of the same layer with its own query
+  if (fused && cfg->plan[cell] == LOOPKV_CELL_REUSE) return LOOPKV_ERR_INVALID_ARG;
   const int src = cfg->plan[cell] == LOOPKV_CELL_REUSE
                       ? (cfg->num_loops - 1) * cfg->num_layers + layer
                       : cell;
@@ -142,11 +150,12 @@ loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const loopkv_cel
   if (len < 0 || len > cap) return LOOPKV_ERR_INVALID_ARG;
   if (len > kMaxSeqLen) return LOOPKV_ERR_UNSUPPORTED;
   if (batch == 0) return LOOPKV_OK;
-  const void* arena = cells->arena[src];
-  const void* residual = cells->key_residual[src];
+  void* arena = cells->arena[src];
+  void* residual = cells->key_residual[src];
   if (!arena || !aligned16(arena)) return LOOPKV_ERR_INVALID_ARG;
   if (kind != LOOPKV_CELL_BF16 && (!residual || !aligned16(residual))) return LOOPKV_ERR_INVALID_ARG;
   if (!q || !aligned16(q) || !out || !block_table || !seq_lens) return LOOPKV_ERR_INVALID_ARG;
+  if (fused && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return LOOPKV_ERR_INVALID_ARG;
 
   const int splits = cfg->decode_splits
                          ? cfg->decode_splits
@@ -170,11 +179,41 @@ loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const loopkv_cel
   p.max_seq_len = len;
   p.tau = tau;
   p.sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.wr_arena = fused ? static_cast<uint8_t*>(arena) : nullptr;
+  p.wr_residual = fused ? static_cast<__nv_bfloat16*>(residual) : nullptr;
   const bool full_values = kind == LOOPKV_CELL_Q4 && tau == 0.f;
   const cudaError_t e = loopkv::launch_decode(kind, cfg->head_dim, p, batch, splits, full_values,
                                               static_cast<cudaStream_t>(stream),
                                               (cfg->flags & LOOPKV_FLAG_PDL) != 0);
   return e == cudaSuccess ? LOOPKV_OK : LOOPKV_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const loopkv_cells* cells,
+                                      int32_t loop, int32_t layer, const void* q,
+                                      const int32_t* block_table, const int32_t* seq_lens,
+                                      int32_t batch, int32_t max_seq_len, float tau,
+                                      float sm_scale, void* out, uint32_t* sel_mask,
+                                      int32_t* sel_count, int32_t* err_flag, void* stream) {
+  return decode_common(cfg, cells, loop, layer, nullptr, nullptr, q, block_table, seq_lens, batch,
+                       max_seq_len, tau, sm_scale, out, sel_mask, sel_count, err_flag, stream);
+}
+
+loopkv_status loopkv_append_decode_attention(const loopkv_config* cfg, const loopkv_cells* cells,
+                                             int32_t loop, int32_t layer, const void* k_new,
+                                             const void* v_new, const void* q,
+                                             const int32_t* block_table, const int32_t* start_pos,
+                                             int32_t batch, int32_t max_seq_len, float tau,
+                                             float sm_scale, void* out, uint32_t* sel_mask,
+                                             int32_t* sel_count, int32_t* err_flag, void* stream) {
+  if (!k_new || !v_new) return LOOPKV_ERR_INVALID_ARG;
+  return decode_common(cfg, cells, loop, layer, k_new, v_new, q, block_table, start_pos, batch,
+                       max_seq_len, tau, sm_scale, out, sel_mask, sel_count, err_flag, stream);
 }
 
 const char* loopkv_status_string(loopkv_status status) {

@@ -60,6 +60,9 @@ def _load():
                                                   VP, VP, I32, I32, VP, VP]),
         "loopkv_decode_attention": (ctypes.c_int, [P(loopkv_config), P(loopkv_cells), I32, I32, VP, VP,
                                                    VP, I32, I32, F32, F32, VP, VP, VP, VP, VP]),
+        "loopkv_append_decode_attention": (ctypes.c_int, [P(loopkv_config), P(loopkv_cells), I32, I32, VP, VP,
+                                                          VP, VP, VP, I32, I32, F32, F32, VP, VP, VP, VP,
+                                                          VP]),
         "loopkv_decode_splits": (I32, [P(loopkv_config), I32, I32, I32]),
         "loopkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
@@ -209,6 +212,30 @@ def loopkv_decode_attention(kv: KVCells, loop: int, layer: int, q, block_table, 
         _ptr(err_flag, "err_flag", torch.int32, optional=True), _stream(stream))
     if st:
         raise LoopKVError(st, "loopkv_decode_attention")
+    return out
+
+
+def loopkv_append_decode_attention(kv: KVCells, loop: int, layer: int, k_new, v_new, q, block_table, start_pos,
+                                   tau: float, sm_scale: float = 1.0, out=None, max_seq_len: int = 0,
+                                   sel_mask=None, sel_count=None, err_flag=None, stream=None):
+    """Append token start_pos[b] (k_new, v_new bf16[B, 1, H, D]) to a stored
+    cell and attend q bf16[B, H, D] over start_pos[b] + 1 tokens, in one
+    launch; returns out bf16[B, H, D]."""
+    if out is None:
+        out = torch.empty_like(q)
+    if k_new.dim() != 4 or k_new.shape[1] != 1:
+        raise ValueError("k_new must be [batch, 1, heads, head_dim]")
+    batch = int(q.shape[0])
+    st = _lib.loopkv_append_decode_attention(
+        ctypes.byref(kv.cfg), ctypes.byref(kv.cells), loop, layer,
+        _ptr(k_new, "k_new", torch.bfloat16), _ptr(v_new, "v_new", torch.bfloat16), _ptr(q, "q", torch.bfloat16),
+        _ptr(block_table, "block_table", torch.int32), _ptr(start_pos, "start_pos", torch.int32),
+        batch, int(max_seq_len), float(tau), float(sm_scale), _ptr(out, "out", torch.bfloat16),
+        _ptr(sel_mask, "sel_mask", torch.int32, optional=True),
+        _ptr(sel_count, "sel_count", torch.int32, optional=True),
+        _ptr(err_flag, "err_flag", torch.int32, optional=True), _stream(stream))
+    if st:
+        raise LoopKVError(st, "loopkv_append_decode_attention")
     return out
 
 

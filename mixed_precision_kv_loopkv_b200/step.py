@@ -18,7 +18,7 @@ from __future__ import annotations
 
 import torch
 
-from .loopkv import (LOOPKV_CELL_REUSE, KVCells, loopkv_decode_attention,
+from .loopkv import (LOOPKV_CELL_REUSE, KVCells, loopkv_append_decode_attention, loopkv_decode_attention,
                      loopkv_quantize_append)
 
 
@@ -47,11 +47,15 @@ class LoopedDecodeStep:
     k_new, v_new : per stored cell, bf16[B, 1, H, D] (None for reuse cells)
     out    : per cell, bf16[B, H, D] (written)
     sel_count : optional per cell int32[B, H] (written)
+    fused  : a stored cell runs append and attention as one launch
+             (loopkv_append_decode_attention); False: two launches
     """
 
     def __init__(self, kv: KVCells, block_table, pos, q, k_new, v_new, out, tau: float,
-                 sm_scale: float, max_seq_len: int, sel_count=None, err_flag=None, cells=None):
+                 sm_scale: float, max_seq_len: int, sel_count=None, err_flag=None, cells=None,
+                 fused: bool = True):
         self.kv = kv
+        self.fused = fused
         self.cells = list(range(len(kv.plan_codes))) if cells is None else sorted(cells)
         self.block_table = block_table
         self.pos = pos
@@ -63,7 +67,7 @@ class LoopedDecodeStep:
 
     def launches_per_step(self) -> int:
         stored = sum(1 for c in self.cells if self.kv.plan_codes[c] != LOOPKV_CELL_REUSE)
-        return len(self.cells) + stored
+        return len(self.cells) + (0 if self.fused else stored)
 
     def run(self, stream=None):
         """Enqueue the step.  Re-running it at the same positions rewrites
@@ -73,6 +77,13 @@ class LoopedDecodeStep:
         for cell in self.cells:
             kind = kv.plan_codes[cell]
             loop, layer = divmod(cell, kv.num_layers)
+            sel = None if self.sel_count is None else self.sel_count[cell]
+            if kind != LOOPKV_CELL_REUSE and self.fused:
+                loopkv_append_decode_attention(kv, loop, layer, self.k_new[cell], self.v_new[cell], self.q[cell],
+                                               self.block_table, self.pos, self.tau, self.sm_scale,
+                                               out=self.out[cell], max_seq_len=self.max_seq_len,
+                                               sel_count=sel, err_flag=self.err_flag, stream=stream)
+                continue
             if kind != LOOPKV_CELL_REUSE:
                 loopkv_quantize_append(kv, loop, layer, self.k_new[cell], self.v_new[cell],
                                        self.block_table, self.pos, err_flag=self.err_flag,

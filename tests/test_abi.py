@@ -32,7 +32,7 @@ def _header_functions():
 
 def test_every_header_function_is_exported(m):
     names = _header_functions()
-    assert len(names) == 7, names
+    assert len(names) == 8, names
     lib = ctypes.CDLL(m.LIB_PATH)
     for name in names:
         assert hasattr(lib, name), name
@@ -167,3 +167,19 @@ def test_split_choice(m):
         assert math.ceil(math.ceil(n / 32) / s) <= 512
     cfg = _cfg(m, [Q4], 1, 1, decode_splits=4)
     assert lib.loopkv_decode_splits(ctypes.byref(cfg), Q4, 2, 64) == 4
+
+
+def _fused(m, cfg, cells, loop=0, layer=0, k=FAKE, v=FAKE, batch=1, tau=0.01):
+    lib = m.library()
+    return lib.loopkv_append_decode_attention(ctypes.byref(cfg), ctypes.byref(cells), loop, layer, k, v, FAKE,
+                                              FAKE, FAKE, batch, 0, tau, 1.0, FAKE, None, None, None, None)
+
+
+def test_fused_step_argument_errors(m):
+    cfg = _cfg(m, [REUSE, Q4], 2, 1)
+    assert _fused(m, cfg, _cells(m, 2), loop=0) == 1          # reuse cells store nothing
+    assert _fused(m, cfg, _cells(m, 2), loop=1, k=None) == 1  # the new token is required
+    assert _fused(m, cfg, _cells(m, 2), loop=1, v=ctypes.c_void_p(0x20008)) == 1
+    assert _fused(m, cfg, _cells(m, 2), loop=1, tau=-1.0) == 1
+    bad = _cfg(m, [Q4, REUSE], 2, 1)
+    assert _fused(m, bad, _cells(m, 2), loop=0) == 2

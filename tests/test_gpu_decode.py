@@ -145,7 +145,7 @@ def test_pdl_flag_matches_plain_launch():
     assert torch.equal(a, b)
 
 
-def _step_parity(name, nseq, cells=None, extra=32):
+def _step_parity(name, nseq, cells=None, extra=32, fused=True):
     """One captured looped decode step (append + attend per cell, PDL,
     CUDA graph) exactly as the benchmark runs it, checked on sampled
     sequences of every cell against the oracle."""
@@ -164,7 +164,8 @@ def _step_parity(name, nseq, cells=None, extra=32):
             kn[c], vn[c] = cell_new_token(w, *divmod(c, w.num_layers), device="cuda")
     pos = lens.clone()
     max_len = int(lens.max()) + extra
-    step = LoopedDecodeStep(kv, table, pos, q, kn, vn, out, w.tau, w.sm_scale, max_len, cells=run_cells)
+    step = LoopedDecodeStep(kv, table, pos, q, kn, vn, out, w.tau, w.sm_scale, max_len, cells=run_cells,
+                            fused=fused)
     step.run()                      # eager warm-up; idempotent at the same position
     torch.cuda.synchronize()
     for c in run_cells:
@@ -193,8 +194,9 @@ def _step_parity(name, nseq, cells=None, extra=32):
     return report
 
 
-def test_ouro_step_captured_with_pdl():
-    rep = _step_parity("ouro_step", nseq=2)
+@pytest.mark.parametrize("fused", [True, False])
+def test_ouro_step_captured_with_pdl(fused):
+    rep = _step_parity("ouro_step", nseq=2, fused=fused)
     assert len(rep) == 96
 
 
