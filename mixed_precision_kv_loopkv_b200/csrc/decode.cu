@@ -731,27 +731,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       table[e] = ent;
     }
   }
-  if constexpr (CLUSTER) cluster_arrive_release();
-
-  // ---- while the splits meet: bring the low-plane rows of this warp's
-  //      candidates into L2.  A token's weight under the global normaliser is
-  //      at most its weight under this warp's own (max, sum), so every token
-  //      pass 2 selects is among these.
-  if (C::kLogits && p.tau > 0.f && p.tau < INFINITY && lw > 0.f) {
-    const float thr = p.tau * lw;
-    for (int gi = warp; gi < cg; gi += kNW) {
-      const float lg = logits[gi * kGroup + lane];
-      if ((g0 + gi) * kGroup + lane < nn && fast_exp2(lg - ws.m) >= thr) {
-        const int phys = ids_smem[2 * gi + (lane >> 4)];
-        if (phys >= 0) {
-          const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
-          prefetch_l2(rec + R::kQ4VLo + (lane & 15) * R::kRow);
-          prefetch_l2(rec + R::kQ4VMeta + (lane & 15) * (D / kGroup) * 4);
-        }
-      }
-    }
-  }
-  if constexpr (CLUSTER) cluster_wait_acquire(); else __syncthreads();
+  if constexpr (CLUSTER) cluster_sync_all(); else __syncthreads();
 
   // ---- global (max, normaliser, errors) from the local table
   float m_g, z;

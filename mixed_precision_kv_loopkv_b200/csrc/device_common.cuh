@@ -150,7 +150,7 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 // Split cluster barrier.  The relaxed arrival at kernel start, waited on
 // before the first store into a peer, proves that every CTA of the cluster
-// has started; release / acquire pairs order the exchanges after it.
+// has started; full barriers (cluster_sync_all) order the exchanges after it.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   __syncwarp();
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -158,14 +158,6 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 __device__ __forceinline__ void cluster_wait() {
   __syncwarp();
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  __syncwarp();
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  __syncwarp();
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
   uint32_t r;
@@ -195,11 +187,6 @@ __device__ __forceinline__ void st_peer_v4(uint32_t addr, float4 v) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y),
                "f"(v.z), "f"(v.w)
                : "memory");
-}
-
-// Hint: bring the line holding p into L2 (no completion, no data returned).
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // ------------------------------------------------ programmatic dependent launch
