@@ -1014,43 +1014,29 @@ long resident_ctas(int kind, int d, int cg, int splits, int sms, int minb) {
 
 }  // namespace
 
-// Largest context one split may hold (its logits live in shared memory).
-constexpr int kMaxGroupsPerSplit = 512;
+// Splits are chosen so that a split holds at most this many groups (its
+// logits buffer stays small enough for four CTAs per SM, and the longest
+// chunk of a ragged batch stays short) ...
+constexpr int kTargetGroupsPerSplit = 160;
 
 int decode_splits(int kind, int head_dim, int batch, int heads, int max_seq_len) {
   const int groups = (max_seq_len + kGroup - 1) / kGroup;
   const long pairs = static_cast<long>(batch) * heads;
-  int min_s = 1;
-  while (min_s < 8 && (groups + min_s - 1) / min_s > kMaxGroupsPerSplit) min_s <<= 1;
-  if (pairs <= 0 || groups <= 1) return min_s;
+  int s = 1;
+  while (s < 8 && (groups + s - 1) / s > kTargetGroupsPerSplit) s <<= 1;
+  if (pairs <= 0 || groups <= 1) return s;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // Score of a split count: for a short grid, the fraction of the resident
-  // slots its waves keep busy; for a long grid (the launch then runs the
-  // 5-per-SM build where that fits more CTAs), busy slots per SM relative to
-  // four, so that more resident warps win once every SM stays loaded.
-  int best = min_s;
-  double best_score = -1.0;
-  for (int s = min_s; s <= 8; s <<= 1) {
-    if (s > min_s && groups < 2 * kNW * s) break;  // keep >= 2 groups per warp
-    const int cg = (groups + s - 1) / s;
-    long slots = resident_ctas(kind, head_dim, cg, s, sms, 4);
+  // ... and, past that, doubled while the grid fills less than 80 % of the
+  // resident slots once (short grids: more, shorter CTAs put every SM to
+  // work), keeping at least two groups per warp
+  while (s < 8 && groups >= 2 * kNW * 2 * s) {
+    long slots = resident_ctas(kind, head_dim, (groups + s - 1) / s, s, sms, 4);
     if (slots <= 0) slots = 4L * sms;  // no device: a fixed guess keeps the choice deterministic
-    const long ctas = pairs * s;
-    const bool long_grid = ctas >= kHighOccupancyWaves * slots;
-    if (long_grid) {
-      const long slots5 = resident_ctas(kind, head_dim, cg, s, sms, 5);
-      if (slots5 > slots) slots = slots5;
-    }
-    const long waves = (ctas + slots - 1) / slots;
-    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
-    const double score = long_grid ? eff * static_cast<double>(slots) / (4.0 * sms) : eff;
-    if (score > best_score + 0.02) {
-      best_score = score;
-      best = s;
-    }
+    if (pairs * s * 5 >= slots * 4) break;
+    s <<= 1;
   }
-  return best;
+  return s;
 }
 
 cudaError_t launch_decode(int kind, int head_dim, const DecodeParams& p, int batch, int splits,
