@@ -163,13 +163,30 @@ def softmax_weights(q, k_hat, sm_scale: float):
     return s, e / e.sum()
 
 
-def select_low_plane(p, tau: float) -> np.ndarray:
-    """Tokens whose fp32 softmax weight is at least tau."""
-    return np.asarray(p, np.float64).astype(np.float32) >= np.float32(tau)
+def select_low_plane(p, tau: float, unit: int = 1) -> np.ndarray:
+    """Tokens whose fp32 softmax weight is at least tau.
+
+    ``unit`` > 1 is the coarser selection granularity the survey lists as a
+    variant of the same rule (16: a paged block, 32: a key group): every
+    token of the aligned unit [u*unit, (u+1)*unit) takes its low plane when
+    the unit's largest fp32 weight is at least tau.
+    """
+    tok = np.asarray(p, np.float64).astype(np.float32) >= np.float32(tau)
+    if unit == 1 or tok.size == 0:
+        return tok
+    if unit not in (16, 32):
+        raise ValueError("selection unit must be 1, 16 or 32")
+    n = tok.size
+    units = -(-n // unit)
+    padded = np.zeros(units * unit, dtype=bool)
+    padded[:n] = tok
+    any_in_unit = padded.reshape(units, unit).any(axis=1)
+    return np.repeat(any_in_unit, unit)[:n]
 
 
-def attend(q, k_hat, v_full, v_high, tau: float, sm_scale: float):
-    """Decode attention of one query.
+def attend(q, k_hat, v_full, v_high, tau: float, sm_scale: float, unit: int = 1):
+    """Decode attention of one query (``unit``: selection granularity, see
+    select_low_plane).
 
     ``v_high`` is None for cells without a low plane (2-bit, bf16); then every
     token uses ``v_full`` and nothing is selected.  Returns (o fp64[D],
@@ -184,7 +201,7 @@ def attend(q, k_hat, v_full, v_high, tau: float, sm_scale: float):
         sel = np.zeros(n, dtype=bool)
         v_hat = np.asarray(v_full, np.float64)
     else:
-        sel = select_low_plane(p, tau)
+        sel = select_low_plane(p, tau, unit)
         v_hat = np.where(sel[:, None], v_full, v_high)
     return p @ v_hat, sel, p
 
@@ -205,14 +222,14 @@ class StoredSequence:
         else:
             raise ValueError(kind)
 
-    def attend(self, q, tau: float, sm_scale: float):
+    def attend(self, q, tau: float, sm_scale: float, unit: int = 1):
         """Attention of one query over every stored token."""
         if self.kind == "bf16":
             return attend(q, self.k_exact, self.v_exact, None, tau, sm_scale)
         k_hat = self.qk.dequant()
         v_full = self.qv.dequant_full()
         v_high = self.qv.dequant_high() if self.kind == "q4" else None
-        return attend(q, k_hat, v_full, v_high, tau, sm_scale)
+        return attend(q, k_hat, v_full, v_high, tau, sm_scale, unit)
 
 
 def resolve_source(plan, cell: int, num_layers: int) -> int:

@@ -221,3 +221,43 @@ def test_high_plane_value_is_bucket_midpoint():
     bucket = np.mean([m + s * (4 * hi + lo) for lo in range(4)], axis=0)
     np.testing.assert_allclose(qv.dequant_high(), bucket, rtol=1e-15, atol=1e-15)
     assert np.all(np.abs(qv.dequant_full() - qv.dequant_high()) <= 1.5 * s + 1e-12)
+
+
+# ---- coarser selection units (the survey's granularity variant): pinned by
+#      brute force over the units, nesting and the decomposition with torch
+
+@pytest.mark.parametrize("unit", [16, 32])
+@pytest.mark.parametrize("n", [1, 15, 16, 33, 517])
+def test_unit_selection_is_any_token_of_the_unit(unit, n):
+    q, k, v, seq = _case(7, n=n, q_scale=3.0)
+    tau = 0.01
+    _, tok, p = seq.attend(q, tau, 1.0)
+    _, sel, _ = seq.attend(q, tau, 1.0, unit=unit)
+    for t in range(n):
+        u0 = (t // unit) * unit
+        assert sel[t] == any(p[i].astype(np.float32) >= np.float32(tau) for i in range(u0, min(n, u0 + unit)))
+    assert np.all(tok <= sel)
+
+
+def test_units_nest_and_reduce_to_tokens():
+    q, k, v, seq = _case(8, n=700, q_scale=4.0)
+    for tau in [1e-3, 1e-2, 5e-2]:
+        s1 = seq.attend(q, tau, 1.0)[1]
+        s16 = seq.attend(q, tau, 1.0, unit=16)[1]
+        s32 = seq.attend(q, tau, 1.0, unit=32)[1]
+        assert np.all(s1 <= s16) and np.all(s16 <= s32)
+        assert s32.sum() <= 32 * math.floor(1 / tau)
+        np.testing.assert_array_equal(s1, seq.attend(q, tau, 1.0, unit=1)[1])
+    for unit in (16, 32):
+        assert seq.attend(q, 0.0, 1.0, unit=unit)[1].all()
+        assert not seq.attend(q, math.inf, 1.0, unit=unit)[1].any()
+
+
+@pytest.mark.parametrize("unit", [16, 32])
+def test_unit_selection_decomposition(unit):
+    q, k, v, seq = _case(9, n=300, q_scale=3.0)
+    o, sel, _ = seq.attend(q, 0.01, 1.0, unit=unit)
+    kh, vf, vh = seq.qk.dequant(), seq.qv.dequant_full(), seq.qv.dequant_high()
+    pt = _torch_p(q, kh, 1.0)
+    ref = _sdpa(q, kh, vh, 1.0) + (pt[sel, None] * (vf - vh)[sel]).sum(axis=0)
+    np.testing.assert_allclose(o, ref, rtol=1e-10, atol=1e-12)
