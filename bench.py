@@ -51,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="ouro_step")
     ap.add_argument("--splits", type=int, default=0, help="decode splits override (0 = automatic)")
     ap.add_argument("--no-pdl", action="store_true")
+    ap.add_argument("--select-unit", type=int, default=1, choices=[1, 16, 32],
+                    help="low-plane selection unit in tokens (1: per token, the method's rule)")
     ap.add_argument("--no-fuse", action="store_true",
                     help="stored cells append and attend in two launches instead of one")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
@@ -199,8 +201,9 @@ def profiled_traffic(workload: str):
 
 # ----------------------------------------------------------------- workload setup
 
-def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0, fused: bool = True):
-    from mixed_precision_kv_loopkv_b200 import LOOPKV_FLAG_PDL, KVCells, LoopedDecodeStep, prefill
+def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0, fused: bool = True, unit: int = 1):
+    from mixed_precision_kv_loopkv_b200 import (LOOPKV_FLAG_PDL, LOOPKV_FLAG_SELECT_BLOCK, LOOPKV_FLAG_SELECT_GROUP,
+                                                KVCells, LoopedDecodeStep, prefill)
     from workload import block_table_for, cell_kv, cell_new_token, cell_query, make_plan, seq_lens_for
 
     plan = make_plan(w)
@@ -212,7 +215,10 @@ def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0, fused: bo
         src = lambda c: c if plan[c] != "reuse" else (w.num_loops - 1) * w.num_layers + c % w.num_layers
         run = sorted(set(range(ncells)) | {src(c) for c in range(ncells)})
     kv = KVCells(plan, w.num_loops, w.num_layers, w.num_heads, w.head_dim, num_blocks, w.batch,
-                 table_np.shape[1], flags=LOOPKV_FLAG_PDL if pdl else 0, decode_splits=splits,
+                 table_np.shape[1],
+                 flags=(LOOPKV_FLAG_PDL if pdl else 0) | {1: 0, 16: LOOPKV_FLAG_SELECT_BLOCK,
+                                                          32: LOOPKV_FLAG_SELECT_GROUP}[unit],
+                 decode_splits=splits,
                  allocate=set(run))
     table = torch.from_numpy(table_np).cuda()
     stored = [c for c in run if plan[c] != "reuse"]
@@ -385,7 +391,8 @@ def main_arm(args, world, rank, local):
     w = get_workload(args.workload)
     if args.batch:
         w = w.with_(batch=args.batch)
-    S = setup(w, pdl=not args.no_pdl, splits=args.splits, ncells=args.cells, fused=not args.no_fuse)
+    S = setup(w, pdl=not args.no_pdl, splits=args.splits, ncells=args.cells, fused=not args.no_fuse,
+              unit=args.select_unit)
     step, plan, lens = S["step"], S["plan"], S["lens"]
     dev = torch.device(f"cuda:{local}")
 
@@ -451,7 +458,7 @@ def main_arm(args, world, rank, local):
         cfg = workload_config(w, world)
         if args.cells:
             cfg["cells_run"] = len(step.cells)
-        cfg.update({"pdl": not args.no_pdl, "fused_append": not args.no_fuse,
+        cfg.update({"pdl": not args.no_pdl, "fused_append": not args.no_fuse, "select_unit": args.select_unit,
                     "splits": args.splits or "auto", "cuda_graph": True,
                     "algorithmic_bytes_per_step": bytes_step,
                     "selected_low_plane_rows_per_step": int(sel.sum())})

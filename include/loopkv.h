@@ -105,6 +105,11 @@ typedef enum {
                                seq_len - 1, before it waits: the previous kernel
                                must not write those (a decode step's append only
                                writes that last group and the key residual). */
+#define LOOPKV_FLAG_SELECT_BLOCK 0x2 /* coarser low-plane selection: every token of
+                               an aligned 16-token block takes its low plane when
+                               the block's largest fp32 weight is >= tau */
+#define LOOPKV_FLAG_SELECT_GROUP 0x4 /* the same over aligned 32-token groups
+                               (at most one of the two selection flags) */
 
 typedef struct {
   int32_t num_loops;          /* L */

@@ -20,6 +20,8 @@ from .loopkv import (  # noqa: F401
     LOOPKV_DEVERR_SEQ_LEN,
     LOOPKV_DEVERR_TIMEOUT,
     LOOPKV_FLAG_PDL,
+    LOOPKV_FLAG_SELECT_BLOCK,
+    LOOPKV_FLAG_SELECT_GROUP,
     KVCells,
     LoopKVError,
     library,

@@ -769,7 +769,17 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       } else {
         sel = C::kQ4 && valid;  // tau = 0: every token took its low plane in pass 1
       }
-      const uint32_t mask = __ballot_sync(0xffffffffu, sel);
+      uint32_t mask = __ballot_sync(0xffffffffu, sel);
+      if (C::kLogits && p.sel_unit > 1) {
+        // coarser units: a 16-token block or the whole group takes its low
+        // plane when any of its tokens reaches tau (groups and blocks align)
+        const uint32_t valid_mask = __ballot_sync(0xffffffffu, valid);
+        if (p.sel_unit == 16)
+          mask = ((mask & 0x0000FFFFu) ? 0x0000FFFFu : 0u) | ((mask & 0xFFFF0000u) ? 0xFFFF0000u : 0u);
+        else
+          mask = mask ? 0xFFFFFFFFu : 0u;
+        mask &= valid_mask;
+      }
       if (lane == 0) {
         if (p.sel_mask) p.sel_mask[(static_cast<size_t>(b) * p.H + h) * p.mask_words + g0 + gi] = mask;
         if constexpr (C::kLogits) masks_smem[gi] = mask;

@@ -34,6 +34,7 @@ struct DecodeParams {
   int max_seq_len;
   float tau;
   float sm_scale_log2;            // sm_scale * log2(e)
+  int sel_unit;                   // low-plane selection unit: 1, 16 or 32 tokens
   // fused append (k_new non-null): seq_lens holds start positions; the
   // kernel first stores token start_pos[b] into the cell, then attends over
   // start_pos[b] + 1 tokens (negative start: sequence skipped)

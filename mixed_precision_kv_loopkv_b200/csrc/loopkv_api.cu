@@ -24,6 +24,8 @@ loopkv_status check_config(const loopkv_config* cfg) {
     return LOOPKV_ERR_INVALID_ARG;
   if (cfg->head_dim != 64 && cfg->head_dim != 128) return LOOPKV_ERR_UNSUPPORTED;
   if (cfg->block_size != 16) return LOOPKV_ERR_UNSUPPORTED;
+  if ((cfg->flags & LOOPKV_FLAG_SELECT_BLOCK) && (cfg->flags & LOOPKV_FLAG_SELECT_GROUP))
+    return LOOPKV_ERR_INVALID_ARG;
   const int s = cfg->decode_splits;
   if (s != 0 && s != 1 && s != 2 && s != 4 && s != 8) return LOOPKV_ERR_INVALID_ARG;
   const int L = cfg->num_loops, N = cfg->num_layers;
@@ -179,6 +181,7 @@ loopkv_status decode_common(const loopkv_config* cfg, const loopkv_cells* cells,
   p.max_seq_len = len;
   p.tau = tau;
   p.sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  p.sel_unit = (cfg->flags & LOOPKV_FLAG_SELECT_BLOCK) ? 16 : (cfg->flags & LOOPKV_FLAG_SELECT_GROUP) ? 32 : 1;
   p.k_new = static_cast<const __nv_bfloat16*>(k_new);
   p.v_new = static_cast<const __nv_bfloat16*>(v_new);
   p.wr_arena = fused ? static_cast<uint8_t*>(arena) : nullptr;

@@ -21,7 +21,7 @@ LOOPKV_CELL_Q4, LOOPKV_CELL_Q2, LOOPKV_CELL_REUSE, LOOPKV_CELL_BF16 = 0, 1, 2, 3
 KIND_CODES = {"q4": LOOPKV_CELL_Q4, "q2": LOOPKV_CELL_Q2, "reuse": LOOPKV_CELL_REUSE,
               "bf16": LOOPKV_CELL_BF16}
 LOOPKV_DEVERR_BLOCK_ID, LOOPKV_DEVERR_SEQ_LEN, LOOPKV_DEVERR_TIMEOUT, LOOPKV_DEVERR_RANGE = 0x1, 0x2, 0x4, 0x8
-LOOPKV_FLAG_PDL = 0x1
+LOOPKV_FLAG_PDL, LOOPKV_FLAG_SELECT_BLOCK, LOOPKV_FLAG_SELECT_GROUP = 0x1, 0x2, 0x4
 STATUS_NAMES = {0: "LOOPKV_OK", 1: "LOOPKV_ERR_INVALID_ARG", 2: "LOOPKV_ERR_BAD_PLAN",
                 3: "LOOPKV_ERR_UNSUPPORTED", 4: "LOOPKV_ERR_CUDA"}
 

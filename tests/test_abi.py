@@ -183,3 +183,8 @@ def test_fused_step_argument_errors(m):
     assert _fused(m, cfg, _cells(m, 2), loop=1, tau=-1.0) == 1
     bad = _cfg(m, [Q4, REUSE], 2, 1)
     assert _fused(m, bad, _cells(m, 2), loop=0) == 2
+
+
+def test_two_selection_units_are_invalid(m):
+    cfg = _cfg(m, [Q4], 1, 1, flags=0x2 | 0x4)
+    assert _decode(m, cfg, _cells(m, 1)) == 1

@@ -242,3 +242,24 @@ def test_bf16_cells_full_shape_sampled():
     out, sm, sc = _decode(kv, 3, q, table, lens, 0.01)
     check_cell(kv, plan, 3, data, q, table, lens, 0.01, 1.0, sample_pairs(w, 2), out=out, sel_mask=sm,
                sel_count=sc)
+
+
+@pytest.mark.parametrize("unit", [16, 32])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("tau", [0.01, 0.05])
+def test_coarser_selection_units(unit, d, tau):
+    """Low-plane selection by 16-token block or 32-token group (the
+    granularity variant): any token of the unit at or above tau upgrades the
+    whole unit."""
+    from mixed_precision_kv_loopkv_b200 import LOOPKV_FLAG_SELECT_BLOCK, LOOPKV_FLAG_SELECT_GROUP
+    w, kv, data, table, lens = _store_ragged("q4", d, RAGGED, heads=2, seed=13)
+    kv.flags = LOOPKV_FLAG_SELECT_BLOCK if unit == 16 else LOOPKV_FLAG_SELECT_GROUP
+    pairs = [(b, h) for b in range(w.batch) for h in range(2)]
+    q = query_for(w, 0, temperature=4.0)
+    out, sm, sc = _decode(kv, 0, q, table, lens, tau)
+    check_cell(kv, ["q4"], 0, data, q, table, lens, tau, 1.0, pairs, out=out, sel_mask=sm, sel_count=sc,
+               unit=unit)
+    assert int(sc.sum()) > 0
+    kv.flags = 0
+    out1, sm1, sc1 = _decode(kv, 0, q, table, lens, tau)
+    assert int(sc.sum()) >= int(sc1.sum())
