@@ -218,6 +218,34 @@ LOOPKV_API loopkv_status loopkv_append_decode_attention(
     int32_t max_seq_len, float tau, float sm_scale, void* out, uint32_t* sel_mask, int32_t* sel_count,
     int32_t* err_flag, void* stream);
 
+/*
+ * Offline plan of every (loop, layer) cell from a synthetic damage table
+ * (host only, no GPU).  The LoopKV abstract describes a planner that picks
+ * 4-bit, 2-bit or reuse per cell to minimise the bytes read per decoded
+ * token under budgets on predicted (additive) damage and storage; the
+ * formulation here is the library's reading:
+ *   damage       : host int32 [L*N][3], the damage of cell (loop*N + layer)
+ *                  stored 4-bit / 2-bit / as a reuse (column 2 of the final
+ *                  loop is ignored: those cells cannot reuse); >= 0
+ *   damage_budget: sum of the chosen damages must not exceed it
+ *   storage_budget: sum of storage in 32-byte units per token-head
+ *                  (4-bit 5, 2-bit 3, reuse 0) must not exceed it
+ *   q4_read_bytes: bytes a 4-bit cell reads per token-head (128 plus the
+ *                  expected low-plane share); 2-bit reads 96; a reuse cell
+ *                  reads what its source (the final loop's cell) reads
+ *   plan_out     : host uint8 [L*N], LOOPKV_CELL_Q4 / _Q2 / _REUSE
+ *   reads_out    : optional host int64, total reads per token-head
+ * The plan minimises total reads; among plans of equal reads it has the
+ * least damage, then the least storage.  Exact (dynamic program over layers
+ * with (damage, storage) states).  Errors: INVALID_ARG for bad sizes,
+ * negative inputs or num_loops > 6; UNSUPPORTED when (damage_budget + 1) x
+ * (storage_budget + 1) x num_layers exceeds 2^25 states; BAD_PLAN when no
+ * plan meets the budgets (plan_out untouched).
+ */
+LOOPKV_API loopkv_status loopkv_plan_cells(int32_t num_loops, int32_t num_layers, const int32_t* damage,
+                                           int32_t damage_budget, int32_t storage_budget,
+                                           int32_t q4_read_bytes, uint8_t* plan_out, int64_t* reads_out);
+
 /* Context splits (CTAs per sequence and head) a decode call over a source
  * cell of the given kind would launch; 0 for invalid arguments. */
 LOOPKV_API int32_t loopkv_decode_splits(const loopkv_config* cfg, int32_t kind, int32_t batch,

@@ -28,6 +28,7 @@ from .loopkv import (  # noqa: F401
     loopkv_append_decode_attention,
     loopkv_decode_attention,
     loopkv_decode_splits,
+    loopkv_plan_cells,
     loopkv_quantize_append,
     loopkv_record_bytes,
     loopkv_status_string,

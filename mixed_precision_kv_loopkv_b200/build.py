@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libloopkv.so")
-SOURCES = ["loopkv_api.cu", "append.cu", "decode.cu"]
+SOURCES = ["loopkv_api.cu", "append.cu", "decode.cu", "planner.cpp"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -50,7 +50,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     build_dir = os.path.join(HERE, "_build")
     os.makedirs(build_dir, exist_ok=True)
     for src in SOURCES:
-        obj = os.path.join(build_dir, src.replace(".cu", ".o"))
+        obj = os.path.join(build_dir, os.path.splitext(src)[0] + ".o")
         cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-Xptxas", "-v" if verbose else "-O3",
                "-c", os.path.join(CSRC, src), "-o", obj]
         subprocess.run(cmd, check=True, stdout=None if verbose else subprocess.DEVNULL,

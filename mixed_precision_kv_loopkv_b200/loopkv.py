@@ -64,6 +64,7 @@ def _load():
                                                           VP, VP, VP, I32, I32, F32, F32, VP, VP, VP, VP,
                                                           VP]),
         "loopkv_decode_splits": (I32, [P(loopkv_config), I32, I32, I32]),
+        "loopkv_plan_cells": (ctypes.c_int, [I32, I32, VP, I32, I32, I32, VP, VP]),
         "loopkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -242,6 +243,25 @@ def loopkv_append_decode_attention(kv: KVCells, loop: int, layer: int, k_new, v_
 def loopkv_decode_splits(kv: KVCells, kind, batch: int, max_seq_len: int) -> int:
     return int(_lib.loopkv_decode_splits(ctypes.byref(kv.cfg), KIND_CODES.get(kind, kind), batch,
                                          max_seq_len))
+
+
+def loopkv_plan_cells(damage, damage_budget: int, storage_budget: int, q4_read_bytes: int = 128):
+    """Plan every (loop, layer) cell from an integer damage table
+    ``damage[loop][layer][choice]`` (choice 0: 4-bit, 1: 2-bit, 2: reuse).
+    Returns (plan as kind names in cell order, total reads per token-head)."""
+    import numpy as np
+    d = np.ascontiguousarray(np.asarray(damage, dtype=np.int32))
+    if d.ndim != 3 or d.shape[2] != 3:
+        raise ValueError("damage must be [num_loops, num_layers, 3]")
+    L, N = int(d.shape[0]), int(d.shape[1])
+    plan = (ctypes.c_uint8 * (L * N))()
+    reads = ctypes.c_int64(0)
+    st = _lib.loopkv_plan_cells(L, N, d.ctypes.data_as(ctypes.c_void_p), int(damage_budget), int(storage_budget),
+                                int(q4_read_bytes), ctypes.cast(plan, ctypes.c_void_p), ctypes.byref(reads))
+    if st:
+        raise LoopKVError(st, "loopkv_plan_cells")
+    names = {v: k for k, v in KIND_CODES.items()}
+    return [names[int(x)] for x in plan], int(reads.value)
 
 
 def mask_words(kv: KVCells) -> int:

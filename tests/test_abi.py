@@ -32,7 +32,7 @@ def _header_functions():
 
 def test_every_header_function_is_exported(m):
     names = _header_functions()
-    assert len(names) == 8, names
+    assert len(names) == 9, names
     lib = ctypes.CDLL(m.LIB_PATH)
     for name in names:
         assert hasattr(lib, name), name
