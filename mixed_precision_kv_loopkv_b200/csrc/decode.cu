@@ -796,9 +796,41 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     if (live && gather) {
       constexpr int kNB = 4;
       float corr[4] = {0.f, 0.f, 0.f, 0.f};
+      // coarser selection units: walk the selected 16-token blocks, loading
+      // every selected row of a block in one round trip
+      for (int gi = warp; p.sel_unit > 1 && cnt > 0 && gi < cg; gi += kNW) {
+        const uint32_t m = masks_smem[gi];
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t bm = (m >> (16 * half)) & 0xFFFFu;
+          const int phys = bm ? ids_smem[2 * gi + half] : -1;
+          if (phys < 0) continue;
+          const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
+          uint32_t lo16[kBlock], mv16[kBlock];
+#pragma unroll
+          for (int t = 0; t < kBlock; ++t) {
+            lo16[t] = mv16[t] = 0u;
+            if (lane < D / 4 && ((bm >> t) & 1u)) {
+              lo16[t] = rec[R::kQ4VLo + t * R::kRow + lane];
+              mv16[t] = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VMeta +
+                                                           (t * (D / kGroup) + (4 * lane) / kGroup) * 4);
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < kBlock; ++t) {
+            if ((bm >> t) & 1u) {
+              const float wsel =
+                  fast_exp2(logits[gi * kGroup + kBlock * half + t] - m_g) * inv_z * bf16_lo(mv16[t]);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                corr[i] = fmaf(wsel, static_cast<float>((lo16[t] >> (2 * i)) & 3u) - 1.5f, corr[i]);
+            }
+          }
+        }
+      }
       int gcur = warp;
-      uint32_t mcur = (cnt > 0 && gcur < cg) ? masks_smem[gcur] : 0u;
-      int left = cnt;
+      uint32_t mcur = (p.sel_unit == 1 && cnt > 0 && gcur < cg) ? masks_smem[gcur] : 0u;
+      int left = p.sel_unit == 1 ? cnt : 0;
       while (left > 0) {
         int tg[kNB], tt[kNB];
 #pragma unroll
