@@ -263,3 +263,32 @@ def test_coarser_selection_units(unit, d, tau):
     kv.flags = 0
     out1, sm1, sc1 = _decode(kv, 0, q, table, lens, tau)
     assert int(sc.sum()) >= int(sc1.sum())
+
+
+@pytest.mark.parametrize("kind", ["q4", "q2"])
+def test_maximum_context(kind):
+    """The largest context the ABI accepts (65536 tokens after the step:
+    2048 groups, 8 splits of 256 groups, the most the split rule produces),
+    with a ragged partner sequence, on the fused decode step."""
+    from mixed_precision_kv_loopkv_b200 import (KVCells, loopkv_append_decode_attention, loopkv_decode_splits,
+                                                prefill)
+    lens = [65535, 40000]
+    w = _custom(kind, 128, [n + 1 for n in lens], heads=2, seed=17)
+    table, nblocks = block_table_for(w, [n + 1 for n in lens])
+    kv = KVCells([kind], 1, 1, 2, 128, nblocks, 2, table.shape[1])
+    k, v = cell_kv(w, 0, 0, device="cuda", n=65536)
+    table_d = torch.from_numpy(table).cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    prefill(kv, 0, 0, k, v, table_d, lens, err_flag=err)
+    assert loopkv_decode_splits(kv, kind, 2, 65536) == 8
+    kn = torch.stack([k[0, 65535], k[1, 40000]]).unsqueeze(1).contiguous()
+    vn = torch.stack([v[0, 65535], v[1, 40000]]).unsqueeze(1).contiguous()
+    q = query_for(w, 0, temperature=4.0)
+    sm, sc = mask_buffers(kv, 2)
+    start = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    out = loopkv_append_decode_attention(kv, 0, 0, kn, vn, q, table_d, start, 0.01, max_seq_len=65536,
+                                         sel_mask=sm, sel_count=sc, err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err) == 0
+    check_cell(kv, [kind], 0, {0: (k, v)}, q, table_d, start + 1, 0.01, 1.0, [(0, 0), (0, 1), (1, 0)],
+               out=out, sel_mask=sm, sel_count=sc)
