@@ -166,8 +166,8 @@ def softmax_weights(q, k_hat, sm_scale: float):
 def select_low_plane(p, tau: float, unit: int = 1) -> np.ndarray:
     """Tokens whose fp32 softmax weight is at least tau.
 
-    ``unit`` > 1 is the coarser selection granularity the survey lists as a
-    variant of the same rule (16: a paged block, 32: a key group): every
+    ``unit`` > 1 is a coarser granularity of the same rule, offered as a
+    variant (16: a paged block, 32: a key group): every
     token of the aligned unit [u*unit, (u+1)*unit) takes its low plane when
     the unit's largest fp32 weight is at least tau.
     """

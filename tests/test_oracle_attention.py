@@ -223,7 +223,7 @@ def test_high_plane_value_is_bucket_midpoint():
     assert np.all(np.abs(qv.dequant_full() - qv.dequant_high()) <= 1.5 * s + 1e-12)
 
 
-# ---- coarser selection units (the survey's granularity variant): pinned by
+# ---- coarser selection units (a granularity variant of the rule): pinned by
 #      brute force over the units, nesting and the decomposition with torch
 
 @pytest.mark.parametrize("unit", [16, 32])
