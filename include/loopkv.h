@@ -4,10 +4,11 @@
  * LoopKV: Loop-Aware KV Cache Compression for Serving Looped Transformers
  * (Abstract): a looped transformer keeps one KV cell per (loop, layer); an
  * offline plan stores each cell as 4-bit, as 2-bit, or as a reuse of the
- * final loop's cell of the same layer.  A 4-bit value is kept as a high-2-bit
- * plane and a low-2-bit plane; during decoding every token's high plane is
- * read and the low plane only where the cell's own attention weights call
- * for 4-bit precision.  A single fused kernel executes the plan.
+ * final loop's cell of the same layer.  A 4-bit value is stored as two
+ * 2-bit planes (its top and bottom bits); a decode step reads the top plane
+ * of every token and the bottom plane only of tokens that the cell's own
+ * query weights heavily enough, and one kernel launch per cell carries out
+ * its planned precision.
  *
  * The abstract leaves the storage format open.  This library fixes it:
  *   - asymmetric quantisation with bf16 scale and minimum; keys per channel
@@ -199,8 +200,8 @@ LOOPKV_API loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const
  * start_pos[b] (one new token per sequence) exactly as loopkv_quantize_append
  * with num_tokens = 1 would, then attends over start_pos[b] + 1 tokens exactly
  * as loopkv_decode_attention would with seq_lens = start_pos + 1.  This is
- * the single fused kernel per cell the LoopKV abstract describes, with the
- * store of the current token folded into it: the split holding the new
+ * one launch per cell, as the LoopKV abstract describes its serving kernel,
+ * with the store of the current token folded in: the split holding the new
  * token writes it before it reads that token's group.
  *
  *   k_new, v_new : device bf16 [batch][1][H][D]

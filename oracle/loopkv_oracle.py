@@ -9,9 +9,9 @@ What it computes, following LoopKV: Loop-Aware KV Cache Compression for
 Serving Looped Transformers (Abstract):
   * every (loop, layer) cell is stored 4-bit, 2-bit, or reuses the final
     loop's cell of the same layer;
-  * a 4-bit code is kept as a high-2-bit plane and a low-2-bit plane; during
-    decoding the high plane of every value is read and the low plane only for
-    tokens whose own attention weight needs full precision.
+  * a 4-bit code is stored as two 2-bit planes (top and bottom bits); a
+    decode step reads the top plane of every value and the bottom plane only
+    for tokens that the cell's own query weights heavily enough.
 
 The pages leave the quantiser and the threshold rule open; this oracle takes
 the readings the library documents:
