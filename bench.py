@@ -303,11 +303,14 @@ def oracle_sample(w, plan, lens, n_pairs: int, seed: int = 0):
         src = cell if plan[cell] != "reuse" else (w.num_loops - 1) * w.num_layers + cell % w.num_layers
         b, h = int(rng.integers(w.batch)), int(rng.integers(w.num_heads))
         n = int(lens[b])
-        k, v = cell_kv(w, *divmod(src, w.num_layers), device="cuda")
+        # the GPU arm's inputs come from the CUDA generator; without a GPU the
+        # CPU generator gives inputs of the same distribution
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        k, v = cell_kv(w, *divmod(src, w.num_layers), device=dev)
         kk = k[b, :n, h].float().cpu().numpy()
         vv = v[b, :n, h].float().cpu().numpy()
         del k, v
-        q = cell_query(w, *divmod(cell, w.num_layers), device="cuda")[b, h].float().cpu().numpy()
+        q = cell_query(w, *divmod(cell, w.num_layers), device=dev)[b, h].float().cpu().numpy()
         items.append((plan[src], O.StoredSequence(plan[src], kk, vv), q, n))
     torch.cuda.empty_cache()
     return items
