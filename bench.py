@@ -182,9 +182,9 @@ def decode_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """Per-launch DRAM bytes of the decode kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
+def profiled_fields(workload: str) -> dict:
+    """Machine-read fields of the committed ncu summary of the decode kernel
+    (empty unless it was taken on the current kernel source)."""
     path = os.path.join(ROOT, "profiles", f"decode_attention_{workload}.md")
     try:
         fields = {}
@@ -192,10 +192,16 @@ def profiled_traffic(workload: str):
             if ":" in line and line.strip().startswith("- "):
                 k, v = line.strip()[2:].split(":", 1)
                 fields[k.strip()] = v.strip().strip("`")
-        if fields.get("source_sha256") != decode_source_hash():
-            return None
-        return float(fields["dram_bytes_per_launch"])
+        return fields if fields.get("source_sha256") == decode_source_hash() else {}
     except Exception:
+        return {}
+
+
+def profiled_traffic(workload: str):
+    """Per-launch DRAM bytes of the decode kernel from the committed ncu summary."""
+    try:
+        return float(profiled_fields(workload)["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
         return None
 
 
@@ -424,6 +430,10 @@ def main_arm(args, world, rank, local):
     achieved = bytes_step / launches / per_launch_s / 1e9
     peak, peak_kind = hbm_peak()
     traffic = profiled_traffic(w.name)
+    try:
+        inst_per_launch = float(profiled_fields(w.name)["warp_instructions_per_launch"])
+    except (KeyError, ValueError):
+        inst_per_launch = None
 
     # end to end: inputs of every step copied in from pinned host memory,
     # outputs copied back, inside the timed region
@@ -476,6 +486,18 @@ def main_arm(args, world, rank, local):
                          "per_launch_us": per_launch_s * 1e6,
                          "bytes_per_launch": bytes_step / launches,
                          "peak_source": f"{peak_kind} hbm_gbs"},
+            # the launches are bound by instruction issue: warp instructions per
+            # second (ncu count per launch / measured launch time) against the
+            # SMs' issue peak (4 schedulers x SMs x the sampled SM clock)
+            "issue_roofline": None if inst_per_launch is None or not clocks.summary().get("sm_mhz") else {
+                "achieved": inst_per_launch / per_launch_s,
+                "peak": 4 * torch.cuda.get_device_properties(dev).multi_processor_count
+                        * clocks.summary()["sm_mhz"] * 1e6,
+                "unit": "warp instructions / s",
+                "frac": inst_per_launch / per_launch_s / (
+                    4 * torch.cuda.get_device_properties(dev).multi_processor_count
+                    * clocks.summary()["sm_mhz"] * 1e6),
+                "warp_instructions_per_launch": inst_per_launch},
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "us_per_step": e2e_ms / e2e_steps * 1e3},
             "gpu_launches": args.steps * step.launches_per_step(),
