@@ -532,6 +532,19 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   const int S = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_allow_dependents();
+  // Speculative block ids: the first 16 iterations' table entries of batch
+  // slot z, for the chunk this split would get from a sequence of the host
+  // bound max_seq_len.  They are used below when the actual sequence and
+  // chunk match (every uniform-length batch), so the first bulk copies do
+  // not wait for the lengths before reading the block table.
+  const int zslot = blockIdx.z;
+  const int ng_spec = (p.max_seq_len + kGroup - 1) / kGroup;
+  const int g0_spec = min(split * ((ng_spec + S - 1) / S), ng_spec);
+  int raw_spec = -1;
+  {
+    const int lb = 2 * (g0_spec + warp + kNW * (lane >> 1)) + (lane & 1);
+    if (lb < p.max_blocks) raw_spec = p.block_table[static_cast<size_t>(zslot) * p.max_blocks + lb];
+  }
   // Clusters are dispatched roughly in launch order; the z-th batch slot
   // takes the sequence of rank z by decreasing length (ties by index), so
   // ragged batches start their longest sequences first.
@@ -576,13 +589,13 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   const uint64_t pol = l2_evict_first_policy();
   const int32_t* btab = p.block_table + static_cast<size_t>(b) * p.max_blocks;
   // block ids of 16 iterations, two per iteration, spread over the lanes
-  auto load_ids = [&](int it0) {
+  auto load_ids = [&](int it0, bool speculated) {
     const int it = it0 + (lane >> 1);
     int id = -1;
     if (it < nit) {
       const int lb = 2 * (g0 + warp + kNW * it) + (lane & 1);
       if (lb < n_blocks) {
-        id = btab[lb];
+        id = speculated ? raw_spec : btab[lb];
         if (id < 0 || id >= p.num_blocks) {
           atomicOr(&cta_i[kSlotBad], LOOPKV_DEVERR_BLOCK_ID);
           id = -1;
@@ -593,14 +606,14 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   };
   // current and next batch of 16 iterations' ids: the next batch is loaded a
   // whole batch ahead, so its latency never stalls the ring
-  int ids = load_ids(0), ids_next = load_ids(16), ids_base = 0;
+  int ids = load_ids(0, b == zslot && g0 == g0_spec), ids_next = load_ids(16, false), ids_base = 0;
   // issue the bulk copies of iteration `it` into its stage (all lanes call)
   auto issue = [&](int it) {
     if (it >= nit) return;
     if (it - ids_base >= 16) {
       ids_base += 16;
       ids = ids_next;
-      ids_next = load_ids(ids_base + 16);
+      ids_next = load_ids(ids_base + 16, false);
     }
     const int id0 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base));
     const int id1 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base) + 1);
