@@ -520,13 +520,15 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   auto wscr_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w); };
   constexpr int kCorrOff = TS * D * 4;  // after the warp's TS x D partial sums
   auto corr_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w + kCorrOff); };
+  // the CTA's per-channel sums in its own scale, after warp 0's corrections
+  float* cacc = reinterpret_cast<float*>(smem + sp.rings + kCorrOff + D * 4);
   int32_t* ids_smem = reinterpret_cast<int32_t*>(smem + sp.ids);
   uint32_t* masks_smem = reinterpret_cast<uint32_t*>(smem + sp.masks);
   float4* table = reinterpret_cast<float4*>(smem + sp.xchg);
   float* red = reinterpret_cast<float*>(smem + sp.xchg + 16 * 8 * kNW);
   int* cnts = reinterpret_cast<int*>(smem + sp.xchg + 16 * 8 * kNW + 4 * D);
   int* cta_i = reinterpret_cast<int*>(smem + sp.scal);
-  static_assert(kCorrOff + D * 4 <= NSW * STAGE, "warp results must fit in an idle ring");
+  static_assert(kCorrOff + 2 * D * 4 <= NSW * STAGE, "warp results must fit in an idle ring");
 
   const int split = blockIdx.x, h = blockIdx.y;
   const int S = gridDim.x;
@@ -733,7 +735,6 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   }
 
   // ---- publish (max, sum, error bits) of this warp into every split's table
-  //      (the error word includes this warp's own flags, set before this read)
   if constexpr (CLUSTER) cluster_wait();  // every CTA of the cluster has started
   {
     const float4 ent = make_float4(ws.m, lw, __int_as_float(cta_i[kSlotBad]), 0.f);
@@ -744,7 +745,31 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       table[e] = ent;
     }
   }
-  if constexpr (CLUSTER) cluster_sync_all(); else __syncthreads();
+  if constexpr (CLUSTER) cluster_arrive_release();
+
+  // ---- while the splits meet: this CTA's share of every channel in its own
+  //      scale 2^-m_c (the warps' sub-group sums, rescaled and added)
+  __syncthreads();  // every warp's partial sums and table entry are in place
+  float m_c = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kNW; ++w) m_c = fmaxf(m_c, table[split * kNW + w].x);
+  for (int c = threadIdx.x; c < D; c += kThreads) {
+    const int kc = c / CW, i = c % CW;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kNW; ++w) {
+      const float mw = table[split * kNW + w].x;
+      if (mw != -INFINITY) {
+        const float* wsc = wscr_of(w) + kc * CW + (i & 3);
+        float sw = 0.f;
+#pragma unroll
+        for (int rr = 0; rr < TS; ++rr) sw += wsc[rr * D + 4 * wscr_piece<CW>(i >> 2, kc, rr)];
+        v = fmaf(fast_exp2(mw - m_c), sw, v);
+      }
+    }
+    cacc[c] = v;
+  }
+  if constexpr (CLUSTER) cluster_wait_acquire(); else __syncthreads();
 
   // ---- global (max, normaliser, errors) from the local table
   float m_g, z;
@@ -901,19 +926,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     const int c = threadIdx.x;
     float v = 0.f;
     if (live) {
-      const int kc = c / CW, i = c % CW;
-#pragma unroll
-      for (int w = 0; w < kNW; ++w) {
-        const float mw = table[split * kNW + w].x;
-        if (mw != -INFINITY) {
-          const float* wsc = wscr_of(w) + kc * CW + (i & 3);
-          float sw = 0.f;
-#pragma unroll
-          for (int rr = 0; rr < TS; ++rr) sw += wsc[rr * D + 4 * wscr_piece<CW>(i >> 2, kc, rr)];
-          v = fmaf(fast_exp2(mw - m_g), sw, v);
-        }
-      }
-      v *= inv_z;
+      if (m_c != -INFINITY) v = cacc[c] * fast_exp2(m_c - m_g) * inv_z;
       if (C::kLogits && gather) {
 #pragma unroll
         for (int w = 0; w < kNW; ++w) v += corr_of(w)[c];

@@ -150,7 +150,7 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 // Split cluster barrier.  The relaxed arrival at kernel start, waited on
 // before the first store into a peer, proves that every CTA of the cluster
-// has started; full barriers (cluster_sync_all) order the exchanges after it.
+// has started; release / acquire pairs order the exchanges after it.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   __syncwarp();
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -158,6 +158,14 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 __device__ __forceinline__ void cluster_wait() {
   __syncwarp();
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  __syncwarp();
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
   uint32_t r;
