@@ -25,6 +25,9 @@ the readings the library documents:
     ``min + scale * (4 * hi + 1.5)``;
   * a token takes the low plane when its softmax weight, rounded to fp32, is
     at least tau (tau = 0 selects every token, tau = +inf none);
+  * grouped queries (several query heads per KV head): a token's low plane
+    is fetched when any head of the group selects it and then serves every
+    head of the group;
   * attention itself is evaluated in fp64.
 
 Byte layout (the oracle's own reading of the record format, used only to
@@ -206,6 +209,35 @@ def attend(q, k_hat, v_full, v_high, tau: float, sm_scale: float, unit: int = 1)
     return p @ v_hat, sel, p
 
 
+def attend_grouped(queries, k_hat, v_full, v_high, tau: float, sm_scale: float, unit: int = 1):
+    """Decode attention of the G query heads that share one KV head.
+
+    Grouped-query form of the low-plane rule (the survey's selection
+    variants; the pages speak of one query per head): the KV head's low plane
+    of a token is fetched when any query head of the group selects it (its own
+    fp32 weight, or its unit's largest one, reaches tau), and a fetched row
+    serves every head of the group.  So each head's values are the full 4-bit
+    values on the union of the heads' selections and the high-plane midpoints
+    elsewhere, while each head keeps its own softmax weights.  Returns
+    (o fp64[G, D], selected bool[n], p fp64[G, n]).
+    """
+    queries = np.asarray(queries, np.float32)
+    g = queries.shape[0]
+    k_hat = np.asarray(k_hat, np.float64)
+    n, d = k_hat.shape
+    if n == 0:
+        return np.zeros((g, d)), np.zeros(0, dtype=bool), np.zeros((g, 0))
+    p = np.stack([softmax_weights(qh, k_hat, sm_scale)[1] for qh in queries])
+    sel = np.zeros(n, dtype=bool)
+    if v_high is None:
+        v_hat = np.asarray(v_full, np.float64)
+    else:
+        for h in range(g):
+            sel |= select_low_plane(p[h], tau, unit)
+        v_hat = np.where(sel[:, None], v_full, v_high)
+    return p @ v_hat, sel, p
+
+
 class StoredSequence:
     """One (stored cell, sequence, head): the quantised (or exact) K and V."""
 
@@ -230,6 +262,14 @@ class StoredSequence:
         v_full = self.qv.dequant_full()
         v_high = self.qv.dequant_high() if self.kind == "q4" else None
         return attend(q, k_hat, v_full, v_high, tau, sm_scale, unit)
+
+    def attend_grouped(self, queries, tau: float, sm_scale: float, unit: int = 1):
+        """Attention of the G query heads sharing this KV head (see
+        attend_grouped)."""
+        if self.kind == "bf16":
+            return attend_grouped(queries, self.k_exact, self.v_exact, None, tau, sm_scale)
+        v_high = self.qv.dequant_high() if self.kind == "q4" else None
+        return attend_grouped(queries, self.qk.dequant(), self.qv.dequant_full(), v_high, tau, sm_scale, unit)
 
 
 def resolve_source(plan, cell: int, num_layers: int) -> int:

@@ -261,3 +261,111 @@ def test_unit_selection_decomposition(unit):
     pt = _torch_p(q, kh, 1.0)
     ref = _sdpa(q, kh, vh, 1.0) + (pt[sel, None] * (vf - vh)[sel]).sum(axis=0)
     np.testing.assert_allclose(o, ref, rtol=1e-10, atol=1e-12)
+
+
+# ---- grouped queries (several query heads per KV head): the low plane of a
+#      token is fetched when any head of the group selects it and then serves
+#      every head.  Pinned by torch's attention per head, brute force over
+#      the heads, the per-head bound |S_h| <= 1/tau and special cases.
+
+def _queries(seed, g, d=128, scale=3.0):
+    rng = np.random.default_rng(seed)
+    return np.stack([_bf16(rng, (d,), scale) for _ in range(g)])
+
+
+@pytest.mark.parametrize("kind", ["q4", "q2", "bf16"])
+def test_grouped_single_head_is_attend(kind):
+    q, k, v, seq = _case(21, n=257, kind=kind, q_scale=3.0)
+    o, sel, p = seq.attend_grouped(q[None], 0.01, 1.0)
+    o1, sel1, p1 = seq.attend(q, 0.01, 1.0)
+    np.testing.assert_array_equal(o[0], o1)
+    np.testing.assert_array_equal(sel, sel1)
+    np.testing.assert_array_equal(p[0], p1)
+
+
+@pytest.mark.parametrize("g", [2, 4, 8])
+@pytest.mark.parametrize("unit", [1, 16, 32])
+def test_grouped_union_decomposition(g, unit):
+    """Each head: torch attention over the high-plane values plus, over the
+    union of the heads' own selections, p_h(t) (full - high); the union is
+    brute-forced token by token from torch's weights."""
+    q, k, v, seq = _case(22, n=300)
+    qs = _queries(23, g)
+    tau = 0.01
+    o, sel, p = seq.attend_grouped(qs, tau, 1.0, unit=unit)
+    kh, vf, vh = seq.qk.dequant(), seq.qv.dequant_full(), seq.qv.dequant_high()
+    pt = [_torch_p(qs[h], kh, 1.0) for h in range(g)]
+    want = np.zeros(300, dtype=bool)
+    for t in range(300):
+        u0 = (t // unit) * unit
+        want[t] = any(np.float32(pt[h][i]) >= np.float32(tau)
+                      for h in range(g) for i in range(u0, min(300, u0 + unit)))
+    np.testing.assert_array_equal(sel, want)
+    for h in range(g):
+        ref = _sdpa(qs[h], kh, vh, 1.0) + (pt[h][sel, None] * (vf - vh)[sel]).sum(axis=0)
+        np.testing.assert_allclose(o[h], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_grouped_brute_force_tiny_loops():
+    """Scalar loops (math.exp, Python floats) over heads, tokens and channels
+    on a tiny 4-bit case with three query heads."""
+    rng = np.random.default_rng(24)
+    n, d, g, tau = 40, 32, 3, 0.04
+    k, v = _bf16(rng, (n, d)), _bf16(rng, (n, d))
+    qs = np.stack([_bf16(rng, (d,), 2.0) for _ in range(g)])
+    seq = O.StoredSequence("q4", k, v)
+    o, sel, _ = seq.attend_grouped(qs, tau, 1.0)
+    qk, qv = seq.qk, seq.qv
+    key = [[(float(qk.minv[0, c]) + float(qk.scale[0, c]) * int(qk.codes[t, c])) if t < 32 else float(k[t, c])
+            for c in range(d)] for t in range(n)]
+    probs = []
+    for h in range(g):
+        logits = [sum(float(qs[h][c]) * key[t][c] for c in range(d)) for t in range(n)]
+        m = max(logits)
+        e = [math.exp(s - m) for s in logits]
+        z = sum(e)
+        probs.append([x / z for x in e])
+    union = [any(np.float32(probs[h][t]) >= np.float32(tau) for h in range(g)) for t in range(n)]
+    assert list(sel) == union
+    for h in range(g):
+        out = [0.0] * d
+        for t in range(n):
+            for c in range(d):
+                code = int(qv.codes[t, c])
+                s, mn = float(qv.scale[t, 0]), float(qv.minv[t, 0])
+                out[c] += probs[h][t] * (mn + s * (code if union[t] else 4 * (code >> 2) + 1.5))
+        np.testing.assert_allclose(o[h], out, rtol=1e-11, atol=1e-13)
+
+
+def test_grouped_special_cases_and_bounds():
+    q, k, v, seq = _case(25, n=400, q_scale=3.0)
+    qs = _queries(26, 4)
+    kh, vf, vh = seq.qk.dequant(), seq.qv.dequant_full(), seq.qv.dequant_high()
+    # tau = 0: full 4-bit values for every head; tau = inf: midpoints
+    o0, s0, _ = seq.attend_grouped(qs, 0.0, 1.0)
+    oi, si, _ = seq.attend_grouped(qs, math.inf, 1.0)
+    assert s0.all() and not si.any()
+    for h in range(4):
+        np.testing.assert_allclose(o0[h], _sdpa(qs[h], kh, vf, 1.0), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(oi[h], _sdpa(qs[h], kh, vh, 1.0), rtol=1e-10, atol=1e-12)
+    for tau in [1e-3, 1e-2, 5e-2]:
+        _, sel, _ = seq.attend_grouped(qs, tau, 1.0)
+        own = [seq.attend(qs[h], tau, 1.0)[1] for h in range(4)]
+        # the union holds every head's own set and at most G / tau tokens
+        assert all(np.all(s <= sel) for s in own)
+        assert sel.sum() <= 4 * math.floor(1 / tau)
+        np.testing.assert_array_equal(sel, np.logical_or.reduce(own))
+    # identical queries: the union is that head's own selection
+    same = np.stack([qs[0]] * 3)
+    o, sel, _ = seq.attend_grouped(same, 0.01, 1.0)
+    o1, sel1, _ = seq.attend(qs[0], 0.01, 1.0)
+    np.testing.assert_array_equal(sel, sel1)
+    for h in range(3):
+        np.testing.assert_array_equal(o[h], o1)
+    # 2-bit and bf16 sources select nothing, whatever the group
+    for kind in ("q2", "bf16"):
+        _, _, _, s2 = _case(25, n=50, kind=kind)
+        assert not s2.attend_grouped(_queries(27, 2), 0.01, 1.0)[1].any()
+    # an empty sequence gives zeros for every head
+    e = O.attend_grouped(qs, np.zeros((0, 128)), np.zeros((0, 128)), np.zeros((0, 128)), 0.01, 1.0)
+    assert e[0].shape == (4, 128) and not e[0].any() and e[1].size == 0

@@ -36,6 +36,11 @@ class Workload:
     outlier_scale: float = 10.0
     q_std: float = 0.125              # q ~ N(0, 1) / 8, already carrying its scale
     sm_scale: float = 1.0
+    num_kv_heads: int = 0             # KV heads (0: one per query head, MHA)
+
+    @property
+    def kv_heads(self) -> int:
+        return self.num_kv_heads or self.num_heads
 
     @property
     def num_cells(self) -> int:

@@ -100,17 +100,17 @@ def block_table_for(w: Workload, capacity_tokens) -> tuple:
 
 def _outlier_scale(w: Workload, loop: int, layer: int) -> torch.Tensor:
     rng = np.random.default_rng([w.seed, loop, layer, _TAG_OUTLIER])
-    scale = np.ones((w.num_heads, w.head_dim), dtype=np.float32)
-    for h in range(w.num_heads):
+    scale = np.ones((w.kv_heads, w.head_dim), dtype=np.float32)
+    for h in range(w.kv_heads):
         ch = rng.choice(w.head_dim, size=min(w.outlier_channels, w.head_dim), replace=False)
         scale[h, ch] = w.outlier_scale
     return torch.from_numpy(scale)
 
 
 def cell_kv(w: Workload, loop: int, layer: int, device="cpu", n: int | None = None):
-    """K, V bf16[B, n, H, D] of one stored cell (n defaults to max_context)."""
+    """K, V bf16[B, n, Hkv, D] of one stored cell (n defaults to max_context)."""
     n = w.max_context if n is None else n
-    shape = (w.batch, n, w.num_heads, w.head_dim)
+    shape = (w.batch, n, w.kv_heads, w.head_dim)
     k = torch.randn(shape, generator=_gen(device, w.seed, loop, layer, _TAG_K), device=device)
     k.mul_(_outlier_scale(w, loop, layer).to(device))
     v = torch.randn(shape, generator=_gen(device, w.seed, loop, layer, _TAG_V), device=device)
@@ -118,8 +118,8 @@ def cell_kv(w: Workload, loop: int, layer: int, device="cpu", n: int | None = No
 
 
 def cell_new_token(w: Workload, loop: int, layer: int, device="cpu", step: int = 0):
-    """K, V bf16[B, 1, H, D] of the token appended at decode step ``step``."""
-    shape = (w.batch, 1, w.num_heads, w.head_dim)
+    """K, V bf16[B, 1, Hkv, D] of the token appended at decode step ``step``."""
+    shape = (w.batch, 1, w.kv_heads, w.head_dim)
     k = torch.randn(shape, generator=_gen(device, w.seed, loop, layer, _TAG_NEWK, step), device=device)
     k.mul_(_outlier_scale(w, loop, layer).to(device))
     v = torch.randn(shape, generator=_gen(device, w.seed, loop, layer, _TAG_NEWV, step), device=device)
