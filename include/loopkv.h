@@ -20,7 +20,7 @@
  *
  * Paged storage (PagedAttention-style blocks, background from the same
  * pages' listing of serving papers): a stored cell owns one arena
- *   uint8 arena[num_blocks][num_heads][record]
+ *   uint8 arena[num_blocks][Hkv][record]     (Hkv = KV heads, see loopkv_config)
  * addressed through a block table int32[batch][max_blocks_per_seq] that maps
  * logical block (token / block_size) to a physical block id.  One record holds
  * block_size (16) tokens of one head:
@@ -115,7 +115,7 @@ typedef enum {
 typedef struct {
   int32_t num_loops;          /* L */
   int32_t num_layers;         /* N (layers of the shared block) */
-  int32_t num_heads;          /* query heads = KV heads (MHA) */
+  int32_t num_heads;          /* query heads H */
   int32_t head_dim;           /* D: 64 or 128 */
   int32_t block_size;         /* tokens per paged block: 16 */
   int32_t num_blocks;         /* physical blocks in every stored cell's arena */
@@ -125,21 +125,25 @@ typedef struct {
   int32_t decode_splits;      /* context splits per (sequence, head) for decode:
                                  0 = automatic, else 1, 2, 4 or 8 */
   const uint8_t* plan;        /* host [L*N] loopkv_cell_kind, cell = loop*N + layer */
+  int32_t num_kv_heads;       /* KV heads Hkv; 0 = num_heads (MHA).  Grouped
+                                 queries: num_heads = G * Hkv with G = 1, 2, 4
+                                 or 8 query heads per KV head; query head h
+                                 reads KV head h / G */
 } loopkv_config;
 
 typedef struct {
   /* host [L*N] arrays of device pointers, indexed like plan; NULL for reuse cells */
-  void* const* arena;        /* uint8 [num_blocks][H][record], 16-byte aligned */
-  void* const* key_residual; /* bf16 [max_batch][H][32][D] for 4/2-bit cells, else NULL */
+  void* const* arena;        /* uint8 [num_blocks][Hkv][record], 16-byte aligned */
+  void* const* key_residual; /* bf16 [max_batch][Hkv][32][D] for 4/2-bit cells, else NULL */
 } loopkv_cells;
 
 /* Bytes of one (block, head) record of a stored cell kind (0 if unsupported). */
 LOOPKV_API size_t loopkv_record_bytes(int32_t head_dim, int32_t block_size, int32_t kind);
 
-/* Bytes of one stored cell's arena: num_blocks * num_heads * record. */
+/* Bytes of one stored cell's arena: num_blocks * Hkv * record. */
 LOOPKV_API size_t loopkv_arena_bytes(const loopkv_config* cfg, int32_t kind);
 
-/* Bytes of one key residual: max_batch * num_heads * 32 * head_dim * 2. */
+/* Bytes of one key residual: max_batch * Hkv * 32 * head_dim * 2. */
 LOOPKV_API size_t loopkv_residual_bytes(const loopkv_config* cfg);
 
 /*
@@ -152,7 +156,7 @@ LOOPKV_API size_t loopkv_residual_bytes(const loopkv_config* cfg);
  * rows unchanged.  A bulk append and the same tokens appended one at a time
  * produce identical arena bytes.
  *
- *   k_new, v_new : device bf16 [batch][num_tokens][H][D]
+ *   k_new, v_new : device bf16 [batch][num_tokens][Hkv][D]
  *   block_table  : device int32 [batch][max_blocks_per_seq]
  *   start_pos    : device int32 [batch]; a negative entry skips that sequence
  *   err_flag     : optional device int32 (LOOPKV_DEVERR_* bits)
@@ -172,6 +176,11 @@ LOOPKV_API loopkv_status loopkv_quantize_append(const loopkv_config* cfg, const 
  * the source cell's precision.  For 4-bit sources, every value contributes its
  * high-plane midpoint; tokens with fp32 softmax weight p >= tau then add their
  * low plane (tau = 0: all tokens, tau = +inf: none).
+ * Grouped queries (G = H / Hkv > 1): the G query heads of a KV head each keep
+ * their own softmax weights, and a token's low plane is fetched when any of
+ * them selects it; it then serves all G heads (their values are full 4-bit
+ * on the union of the heads' selections).  sel_mask and sel_count report
+ * that union for every head of the group.
  *
  *   q           : device bf16 [batch][H][D]
  *   block_table : device int32 [batch][max_blocks_per_seq]
@@ -186,7 +195,10 @@ LOOPKV_API loopkv_status loopkv_quantize_append(const loopkv_config* cfg, const 
  *   sel_count   : optional device int32 [batch][H], number of selected tokens
  *   err_flag    : optional device int32
  * Errors: INVALID_ARG for tau < 0 or NaN, null required pointers, batch
- * outside [0, max_batch]; BAD_PLAN; UNSUPPORTED for max_seq_len above 65536.
+ * outside [0, max_batch]; BAD_PLAN; UNSUPPORTED for max_seq_len above 65536,
+ * for a 4-bit source with G x decode_splits above 8 (the CTAs of one KV
+ * head's query heads and splits form one thread-block cluster), or for a
+ * context split too long for one CTA's shared memory.
  */
 LOOPKV_API loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const loopkv_cells* cells,
                                       int32_t loop, int32_t layer, const void* q,
@@ -204,13 +216,14 @@ LOOPKV_API loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const
  * with the store of the current token folded in: the split holding the new
  * token writes it before it reads that token's group.
  *
- *   k_new, v_new : device bf16 [batch][1][H][D]
+ *   k_new, v_new : device bf16 [batch][1][Hkv][D]
  *   start_pos    : device int32 [batch]; a negative entry skips that sequence
  *                  (nothing stored, zeros out)
  *   max_seq_len  : host upper bound on start_pos + 1; 0 means the capacity
  *   other arguments as for loopkv_decode_attention
- * Errors: as loopkv_decode_attention, and INVALID_ARG for a reuse cell or
- * null k_new / v_new.  Device faults: LOOPKV_DEVERR_SEQ_LEN for start_pos + 1
+ * Errors: as loopkv_decode_attention, INVALID_ARG for a reuse cell or
+ * null k_new / v_new, and UNSUPPORTED with grouped queries (G > 1: append
+ * with loopkv_quantize_append, then decode).  Device faults: LOOPKV_DEVERR_SEQ_LEN for start_pos + 1
  * above max_seq_len or the capacity, BLOCK_ID, RANGE as for the append.
  */
 LOOPKV_API loopkv_status loopkv_append_decode_attention(
@@ -247,8 +260,9 @@ LOOPKV_API loopkv_status loopkv_plan_cells(int32_t num_loops, int32_t num_layers
                                            int32_t damage_budget, int32_t storage_budget,
                                            int32_t q4_read_bytes, uint8_t* plan_out, int64_t* reads_out);
 
-/* Context splits (CTAs per sequence and head) a decode call over a source
- * cell of the given kind would launch; 0 for invalid arguments. */
+/* Context splits (CTAs per sequence and query head) a decode call over a
+ * source cell of the given kind would launch; 0 for invalid arguments or an
+ * unsupported split. */
 LOOPKV_API int32_t loopkv_decode_splits(const loopkv_config* cfg, int32_t kind, int32_t batch,
                              int32_t max_seq_len);
 

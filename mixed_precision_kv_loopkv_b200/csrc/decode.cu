@@ -186,7 +186,7 @@ __device__ __forceinline__ int sequence_of_rank(const int32_t* seq_lens, int B, 
   return __reduce_max_sync(0xffffffffu, found);
 }
 
-// The decode step's append of one token at position pos into (b, h), run by
+// The decode step's append of one token at position pos into (b, KV head h), run by
 // every thread of the CTA that holds the token's group: the value row (both
 // planes and meta) from v_new; the key either joins the exact residual or,
 // as its group's 32nd token, completes the group, which is then quantised
@@ -194,10 +194,10 @@ __device__ __forceinline__ int sequence_of_rank(const int32_t* seq_lens, int B, 
 template <int KIND, int D>
 __device__ __forceinline__ void append_token(const DecodeParams& p, int b, int h, int pos, int warp, int lane) {
   using R = Rec<KIND, D>;
-  const CellRows cell{p.wr_arena, p.block_table + static_cast<size_t>(b) * p.max_blocks, p.err, p.H, h,
+  const CellRows cell{p.wr_arena, p.block_table + static_cast<size_t>(b) * p.max_blocks, p.err, p.Hkv, h,
                       p.max_blocks, p.num_blocks};
-  const __nv_bfloat16* kb = p.k_new + (static_cast<size_t>(b) * p.H + h) * D;
-  const __nv_bfloat16* vb = p.v_new + (static_cast<size_t>(b) * p.H + h) * D;
+  const __nv_bfloat16* kb = p.k_new + (static_cast<size_t>(b) * p.Hkv + h) * D;
+  const __nv_bfloat16* vb = p.v_new + (static_cast<size_t>(b) * p.Hkv + h) * D;
   uint8_t* rec = record_at<KIND, D>(cell, pos);
   const int row = pos % kBlock;
   if constexpr (KIND == LOOPKV_CELL_BF16) {
@@ -210,7 +210,7 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, int b, int h
     }
   } else {
     if (warp < D / kGroup) store_value_group<KIND, D>(rec, row, warp, __bfloat162float(vb[warp * kGroup + lane]), lane, p.err);
-    __nv_bfloat16* res = p.wr_residual + (static_cast<size_t>(b) * p.H + h) * kGroup * D;
+    __nv_bfloat16* res = p.wr_residual + (static_cast<size_t>(b) * p.Hkv + h) * kGroup * D;
     if (pos % kGroup == kGroup - 1) {
       store_key_group<KIND, D>(cell, pos / kGroup, lane == kGroup - 1 ? kb : res + lane * D, warp, lane, kNW);
     } else if (static_cast<int>(threadIdx.x) < D * 2 / 16) {
@@ -507,7 +507,9 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
 
 // MINB: CTAs per SM the register budget is cut for (4: 128 registers per
 // thread; 5: 102, for grids of many waves where occupancy pays).
-template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB>
+// GQ: grouped queries (2^g_log2 > 1 query heads per KV head); the build for
+// one query per KV head carries none of their index arithmetic.
+template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB, bool GQ>
 __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodeParams p) {
   using C = Cfg<KIND, D, FULLV>;
   using R = typename C::R;
@@ -530,8 +532,17 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   int* cta_i = reinterpret_cast<int*>(smem + sp.scal);
   static_assert(kCorrOff + 2 * D * 4 <= NSW * STAGE, "warp results must fit in an idle ring");
 
-  const int split = blockIdx.x, h = blockIdx.y;
+  const int split = blockIdx.x;
   const int S = gridDim.x;
+  // KV head of this CTA's query head blockIdx.y (G = 2^g_log2 query heads
+  // per KV head); with grouped queries the query head itself is read again
+  // after pass 1, so that only one of the two stays live through it
+  const int hk = GQ ? static_cast<int>(blockIdx.y) >> p.g_log2 : static_cast<int>(blockIdx.y);
+  const int Hkv = GQ ? p.Hkv : p.H;
+  // Grouped queries with a low-plane selection: the CTAs of the G query
+  // heads of one KV head (and all their splits) form one cluster of S x G,
+  // rank split + S * (h % G), so that the heads can merge their selections.
+  constexpr bool head_cl = GQ && CLUSTER && C::kLogits;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_allow_dependents();
   // Speculative block ids: the first 16 iterations' table entries of batch
@@ -574,6 +585,10 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     fence_mbar_init();
   }
   if (threadIdx.x == 0) cta_i[kSlotBad] = bad;
+  // the heads of a group OR their selections into every member's words
+  // after the exchange barrier below, which orders these zeros before them
+  if (head_cl)
+    for (int i = threadIdx.x; i < p.chunk_groups; i += kThreads) masks_smem[i] = 0u;
   __syncthreads();
   if constexpr (CLUSTER) cluster_arrive_relaxed();
 
@@ -630,9 +645,9 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       const uint32_t bytes = (id0 >= 0 ? LOAD : 0) + (id1 >= 0 ? LOAD : 0);
       mbar_arrive_expect_tx(bar, bytes);
       if (id0 >= 0)
-        bulk_load(dst, p.arena + (static_cast<size_t>(id0) * p.H + h) * R::kBytes, LOAD, bar, pol);
+        bulk_load(dst, p.arena + (static_cast<size_t>(id0) * Hkv + hk) * R::kBytes, LOAD, bar, pol);
       if (id1 >= 0)
-        bulk_load(dst + C::kHalf, p.arena + (static_cast<size_t>(id1) * p.H + h) * R::kBytes, LOAD, bar, pol);
+        bulk_load(dst + C::kHalf, p.arena + (static_cast<size_t>(id1) * Hkv + hk) * R::kBytes, LOAD, bar, pol);
     }
   };
 
@@ -645,7 +660,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     // the split holding the new token stores it first; its copies of the
     // newest group are issued after the writes are visible to the bulk copies
     if (!bad && nn > 0 && (nn - 1) / kGroup >= g0 && (nn - 1) / kGroup < g0 + cg) {
-      append_token<KIND, D>(p, b, h, nn - 1, warp, lane);
+      append_token<KIND, D>(p, b, hk, nn - 1, warp, lane);
       fence_proxy_async_global();
     }
     __syncthreads();
@@ -658,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     float* qconst = reinterpret_cast<float*>(smem + sp.qconst);
     float* q2buf = reinterpret_cast<float*>(smem + sp.q2buf) + warp * 128;
     for (int c = lane; c < D; c += 32) {
-      const float qv = __bfloat162float(p.q[(static_cast<size_t>(b) * p.H + h) * D + c]) * p.sm_scale_log2;
+      const float qv = __bfloat162float(p.q[(static_cast<size_t>(b) * p.H + blockIdx.y) * D + c]) * p.sm_scale_log2;
       const int i = c & 15;
       // every warp writes the same values: no cross-warp ordering is needed
       qconst[c] = qv;
@@ -671,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
 #pragma unroll
       for (int i = 0; i < CW; ++i) qfr[i] = qconst[CW * k + i];
     }
-    const __nv_bfloat16* res = C::kQuant ? p.residual + (static_cast<size_t>(b) * p.H + h) * kGroup * D : nullptr;
+    const __nv_bfloat16* res = C::kQuant ? p.residual + (static_cast<size_t>(b) * Hkv + hk) * kGroup * D : nullptr;
 
     for (int it = 0; it < nit; ++it) {
       const int stage = it % NSW;
@@ -734,13 +749,17 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
           make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
   }
 
+  const int h = GQ ? cta_id_y() : hk;  // query head
+  const int HC = head_cl ? 1 << p.g_log2 : 1;
+  const int rbase = S * (h & (HC - 1));  // cluster rank of this head's split 0
+
   // ---- publish (max, sum, error bits) of this warp into every split's table
   if constexpr (CLUSTER) cluster_wait();  // every CTA of the cluster has started
   {
     const float4 ent = make_float4(ws.m, lw, __int_as_float(cta_i[kSlotBad]), 0.f);
     const int e = split * kNW + warp;
     if constexpr (CLUSTER) {
-      if (lane < S) st_peer_v4(peer_addr(smem_addr(table + e), lane), ent);
+      if (lane < S) st_peer_v4(peer_addr(smem_addr(table + e), rbase + lane), ent);
     } else if (lane == 0) {
       table[e] = ent;
     }
@@ -818,11 +837,29 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
           mask = mask ? 0xFFFFFFFFu : 0u;
         mask &= valid_mask;
       }
+      if (HC > 1) {
+        // into the same split of every head of the group (itself included)
+        if (lane < HC && mask) or_peer_u32(peer_addr(smem_addr(masks_smem + gi), split + S * lane), mask);
+        continue;
+      }
       if (lane == 0) {
         if (p.sel_mask) p.sel_mask[(static_cast<size_t>(b) * p.H + h) * p.mask_words + g0 + gi] = mask;
         if constexpr (C::kLogits) masks_smem[gi] = mask;
       }
       cnt += __popc(mask);
+    }
+  }
+  if (C::kLogits && HC > 1) {
+    // every head of the group has merged its selection: the union, which
+    // every head gathers and reports
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    if (live && (gather || want_mask)) {
+      for (int gi = warp; gi < cg; gi += kNW) {
+        const uint32_t mask = masks_smem[gi];
+        if (lane == 0 && p.sel_mask) p.sel_mask[(static_cast<size_t>(b) * p.H + h) * p.mask_words + g0 + gi] = mask;
+        cnt += __popc(mask);
+      }
     }
   }
   __syncwarp();  // lane 0's selection words are read by the whole warp below
@@ -843,7 +880,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
           const uint32_t bm = (m >> (16 * half)) & 0xFFFFu;
           const int phys = bm ? ids_smem[2 * gi + half] : -1;
           if (phys < 0) continue;
-          const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
+          const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * Hkv + hk) * R::kBytes;
           uint32_t lo16[kBlock], mv16[kBlock];
 #pragma unroll
           for (int t = 0; t < kBlock; ++t) {
@@ -897,7 +934,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
             const int phys = ids_smem[2 * tg[j] + (tt[j] >> 4)];
             lgv[j] = logits[tg[j] * kGroup + tt[j]];
             if (phys >= 0 && lane < D / 4) {
-              const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * p.H + h) * R::kBytes;
+              const uint8_t* rec = p.arena + (static_cast<size_t>(phys) * Hkv + hk) * R::kBytes;
               mv[j] = *reinterpret_cast<const uint32_t*>(rec + R::kQ4VMeta +
                                                          ((tt[j] & 15) * (D / kGroup) + (4 * lane) / kGroup) * 4);
               lo[j] = rec[R::kQ4VLo + (tt[j] & 15) * R::kRow + lane];
@@ -933,14 +970,14 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       }
     }
     const int slot = split * per_rank + c % per_rank;
-    if constexpr (CLUSTER) st_peer_f32(peer_addr(smem_addr(red + slot), c / per_rank), v);
+    if constexpr (CLUSTER) st_peer_f32(peer_addr(smem_addr(red + slot), rbase + c / per_rank), v);
     else red[slot] = v;
   }
   if (threadIdx.x == 0) {
     int total = 0;
 #pragma unroll
     for (int w = 0; w < kNW; ++w) total += cta_i[kSlotCnt0 + w];
-    if constexpr (CLUSTER) st_peer_s32(peer_addr(smem_addr(cnts + split), 0), total);
+    if constexpr (CLUSTER) st_peer_s32(peer_addr(smem_addr(cnts + split), rbase), total);
     else cnts[split] = total;
   }
   // after this barrier no CTA touches another's shared memory
@@ -969,12 +1006,12 @@ size_t smem_bytes_t(int cg) {
 }
 
 // CTAs of this instantiation that can be resident at once on the device
-// (for clusters: co-resident clusters times the cluster size).
-template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB>
-long resident_ctas_t(int cg, int splits, int sms) {
+// (for clusters of splits x hc: co-resident clusters times the cluster size).
+template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB, bool GQ = false>
+long resident_ctas_t(int cg, int splits, int hc, int sms) {
   const size_t smem = smem_bytes_t<KIND, D, FULLV>(cg);
   if (smem > 227u * 1024u) return 0;
-  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB>;
+  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return 0;
   if (!CLUSTER) {
@@ -983,26 +1020,26 @@ long resident_ctas_t(int cg, int splits, int sms) {
     return static_cast<long>(blocks) * sms;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(splits, 1, 1);
+  cfg.gridDim = dim3(splits, hc, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
   attr.val.clusterDim.x = splits;
-  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.y = hc;
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   int clusters = 0;
   if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return 0;
-  return static_cast<long>(clusters) * splits;
+  return static_cast<long>(clusters) * splits * hc;
 }
 
-template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB>
-cudaError_t launch_t(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
+template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB, bool GQ>
+cudaError_t launch_t(const DecodeParams& p, int batch, int splits, int hc, cudaStream_t stream, bool pdl) {
   const size_t smem = smem_bytes_t<KIND, D, FULLV>(p.chunk_groups);
   if (smem > 227u * 1024u) return cudaErrorInvalidValue;
-  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB>;
+  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -1015,7 +1052,7 @@ cudaError_t launch_t(const DecodeParams& p, int batch, int splits, cudaStream_t 
   if (CLUSTER) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
     attr[na].val.clusterDim.x = splits;
-    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.y = hc;
     attr[na].val.clusterDim.z = 1;
     ++na;
   }
@@ -1030,9 +1067,9 @@ cudaError_t launch_t(const DecodeParams& p, int batch, int splits, cudaStream_t 
 }
 
 template <int KIND, int D, bool FULLV, int MINB>
-long resident_m(int cg, int splits, int sms) {
-  return splits > 1 ? resident_ctas_t<KIND, D, FULLV, true, MINB>(cg, splits, sms)
-                    : resident_ctas_t<KIND, D, FULLV, false, MINB>(cg, splits, sms);
+long resident_m(int cg, int splits, int hc, int sms) {
+  return splits * hc > 1 ? resident_ctas_t<KIND, D, FULLV, true, MINB>(cg, splits, hc, sms)
+                         : resident_ctas_t<KIND, D, FULLV, false, MINB>(cg, splits, 1, sms);
 }
 
 // A grid of at least this many waves of 4-per-SM residency runs the
@@ -1044,38 +1081,44 @@ template <int KIND, int D, bool FULLV>
 cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  (void)sms;
+  const int hc = head_cluster(KIND, 1 << p.g_log2, FULLV);
+  if (splits * hc > 8) return cudaErrorInvalidValue;
+  const bool cl = splits * hc > 1;
+  // grouped queries: one build, at four CTAs per SM
+  if (p.g_log2 > 0)
+    return cl ? launch_t<KIND, D, FULLV, true, 4, true>(p, batch, splits, hc, stream, pdl)
+              : launch_t<KIND, D, FULLV, false, 4, true>(p, batch, splits, 1, stream, pdl);
   if constexpr (KIND != LOOPKV_CELL_BF16 && !FULLV) {
     const long ctas = static_cast<long>(batch) * p.H * splits;
-    const long slots4 = resident_m<KIND, D, FULLV, 4>(p.chunk_groups, splits, sms);
+    const long slots4 = resident_m<KIND, D, FULLV, 4>(p.chunk_groups, splits, 1, sms);
     if (slots4 > 0 && ctas >= kHighOccupancyWaves * slots4 &&
-        resident_m<KIND, D, FULLV, 5>(p.chunk_groups, splits, sms) > slots4)
-      return splits > 1 ? launch_t<KIND, D, FULLV, true, 5>(p, batch, splits, stream, pdl)
-                        : launch_t<KIND, D, FULLV, false, 5>(p, batch, splits, stream, pdl);
+        resident_m<KIND, D, FULLV, 5>(p.chunk_groups, splits, 1, sms) > slots4)
+      return cl ? launch_t<KIND, D, FULLV, true, 5, false>(p, batch, splits, 1, stream, pdl)
+                : launch_t<KIND, D, FULLV, false, 5, false>(p, batch, splits, 1, stream, pdl);
   }
-  return splits > 1 ? launch_t<KIND, D, FULLV, true, 4>(p, batch, splits, stream, pdl)
-                    : launch_t<KIND, D, FULLV, false, 4>(p, batch, splits, stream, pdl);
+  return cl ? launch_t<KIND, D, FULLV, true, 4, false>(p, batch, splits, 1, stream, pdl)
+            : launch_t<KIND, D, FULLV, false, 4, false>(p, batch, splits, 1, stream, pdl);
 }
 
 // Co-resident CTAs of one decode build (0 without a device); minb 5 only
 // exists for the 4-bit and 2-bit kinds.
-long resident_ctas(int kind, int d, int cg, int splits, int sms, int minb) {
+long resident_ctas(int kind, int d, int cg, int splits, int hc, int sms, int minb) {
   if (minb == 5) {
     switch (kind * 1000 + d) {
-      case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 5>(cg, splits, sms);
-      case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 5>(cg, splits, sms);
-      case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 5>(cg, splits, sms);
-      case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 5>(cg, splits, sms);
+      case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 5>(cg, splits, hc, sms);
+      case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 5>(cg, splits, hc, sms);
+      case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 5>(cg, splits, 1, sms);
+      case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 5>(cg, splits, 1, sms);
       default: return 0;
     }
   }
   switch (kind * 1000 + d) {
-    case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 4>(cg, splits, sms);
-    case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 4>(cg, splits, sms);
-    case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 4>(cg, splits, sms);
-    case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 4>(cg, splits, sms);
-    case LOOPKV_CELL_BF16 * 1000 + 128: return resident_m<LOOPKV_CELL_BF16, 128, false, 4>(cg, splits, sms);
-    case LOOPKV_CELL_BF16 * 1000 + 64: return resident_m<LOOPKV_CELL_BF16, 64, false, 4>(cg, splits, sms);
+    case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 4>(cg, splits, hc, sms);
+    case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 4>(cg, splits, hc, sms);
+    case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 4>(cg, splits, 1, sms);
+    case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 4>(cg, splits, 1, sms);
+    case LOOPKV_CELL_BF16 * 1000 + 128: return resident_m<LOOPKV_CELL_BF16, 128, false, 4>(cg, splits, 1, sms);
+    case LOOPKV_CELL_BF16 * 1000 + 64: return resident_m<LOOPKV_CELL_BF16, 64, false, 4>(cg, splits, 1, sms);
     default: return 0;
   }
 }
@@ -1087,24 +1130,41 @@ long resident_ctas(int kind, int d, int cg, int splits, int sms, int minb) {
 // chunk of a ragged batch stays short) ...
 constexpr int kTargetGroupsPerSplit = 160;
 
-int decode_splits(int kind, int head_dim, int batch, int heads, int max_seq_len) {
+int decode_splits(int kind, int head_dim, int batch, int heads, int max_seq_len, int hc) {
   const int groups = (max_seq_len + kGroup - 1) / kGroup;
   const long pairs = static_cast<long>(batch) * heads;
+  const int smax = max_splits(hc);
   int s = 1;
-  while (s < 8 && (groups + s - 1) / s > kTargetGroupsPerSplit) s <<= 1;
+  while (s < smax && (groups + s - 1) / s > kTargetGroupsPerSplit) s <<= 1;
   if (pairs <= 0 || groups <= 1) return s;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // ... and, past that, doubled while the grid fills less than 80 % of the
   // resident slots once (short grids: more, shorter CTAs put every SM to
   // work), keeping at least two groups per warp
-  while (s < 8 && groups >= 2 * kNW * 2 * s) {
-    long slots = resident_ctas(kind, head_dim, (groups + s - 1) / s, s, sms, 4);
+  while (s < smax && groups >= 2 * kNW * 2 * s) {
+    long slots = resident_ctas(kind, head_dim, (groups + s - 1) / s, s, hc, sms, 4);
     if (slots <= 0) slots = 4L * sms;  // no device: a fixed guess keeps the choice deterministic
     if (pairs * s * 5 >= slots * 4) break;
     s <<= 1;
   }
   return s;
+}
+
+size_t decode_smem_bytes(int kind, int head_dim, bool full_values, int chunk_groups) {
+  switch (kind * 1000 + head_dim) {
+    case LOOPKV_CELL_Q4 * 1000 + 128:
+      return full_values ? smem_bytes_t<LOOPKV_CELL_Q4, 128, true>(chunk_groups)
+                         : smem_bytes_t<LOOPKV_CELL_Q4, 128, false>(chunk_groups);
+    case LOOPKV_CELL_Q4 * 1000 + 64:
+      return full_values ? smem_bytes_t<LOOPKV_CELL_Q4, 64, true>(chunk_groups)
+                         : smem_bytes_t<LOOPKV_CELL_Q4, 64, false>(chunk_groups);
+    case LOOPKV_CELL_Q2 * 1000 + 128: return smem_bytes_t<LOOPKV_CELL_Q2, 128, false>(chunk_groups);
+    case LOOPKV_CELL_Q2 * 1000 + 64: return smem_bytes_t<LOOPKV_CELL_Q2, 64, false>(chunk_groups);
+    case LOOPKV_CELL_BF16 * 1000 + 128: return smem_bytes_t<LOOPKV_CELL_BF16, 128, false>(chunk_groups);
+    case LOOPKV_CELL_BF16 * 1000 + 64: return smem_bytes_t<LOOPKV_CELL_BF16, 64, false>(chunk_groups);
+    default: return 0;
+  }
 }
 
 cudaError_t launch_decode(int kind, int head_dim, const DecodeParams& p, int batch, int splits,

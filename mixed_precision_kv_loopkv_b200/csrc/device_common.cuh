@@ -135,6 +135,14 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// blockIdx.y read afresh (not merged with earlier reads, so that it need not
+// stay in a register in between)
+__device__ __forceinline__ int cta_id_y() {
+  int r;
+  asm volatile("mov.u32 %0, %%ctaid.y;" : "=r"(r));
+  return r;
+}
+
 // ----------------------------------------------------------------- cluster
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -195,6 +203,11 @@ __device__ __forceinline__ void st_peer_v4(uint32_t addr, float4 v) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y),
                "f"(v.z), "f"(v.w)
                : "memory");
+}
+// Atomic OR into a word of a cluster CTA's shared memory (this CTA's own
+// included); visible after the next release / acquire cluster barrier.
+__device__ __forceinline__ void or_peer_u32(uint32_t addr, uint32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.or.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 // ------------------------------------------------ programmatic dependent launch

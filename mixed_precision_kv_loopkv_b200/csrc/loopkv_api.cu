@@ -10,8 +10,12 @@
 namespace {
 
 constexpr int kMaxSeqLen = 65536;
+constexpr size_t kMaxSmemPerCta = 227u * 1024u;  // opt-in dynamic shared memory of one CTA
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// KV heads of a config (0 in num_kv_heads: one per query head).
+int kv_heads(const loopkv_config* cfg) { return cfg->num_kv_heads ? cfg->num_kv_heads : cfg->num_heads; }
 
 bool stored_kind(int k) {
   return k == LOOPKV_CELL_Q4 || k == LOOPKV_CELL_Q2 || k == LOOPKV_CELL_BF16;
@@ -22,6 +26,9 @@ loopkv_status check_config(const loopkv_config* cfg) {
   if (cfg->num_loops <= 0 || cfg->num_layers <= 0 || cfg->num_heads <= 0 || cfg->num_blocks < 0 ||
       cfg->max_batch < 0 || cfg->max_blocks_per_seq <= 0)
     return LOOPKV_ERR_INVALID_ARG;
+  if (cfg->num_kv_heads < 0 || cfg->num_heads % kv_heads(cfg) != 0) return LOOPKV_ERR_INVALID_ARG;
+  const int group = cfg->num_heads / kv_heads(cfg);  // query heads per KV head: 1, 2, 4 or 8
+  if (group != 1 && group != 2 && group != 4 && group != 8) return LOOPKV_ERR_UNSUPPORTED;
   if (cfg->head_dim != 64 && cfg->head_dim != 128) return LOOPKV_ERR_UNSUPPORTED;
   if (cfg->block_size != 16) return LOOPKV_ERR_UNSUPPORTED;
   if ((cfg->flags & LOOPKV_FLAG_SELECT_BLOCK) && (cfg->flags & LOOPKV_FLAG_SELECT_GROUP))
@@ -62,14 +69,14 @@ size_t loopkv_record_bytes(int32_t head_dim, int32_t block_size, int32_t kind) {
 }
 
 size_t loopkv_arena_bytes(const loopkv_config* cfg, int32_t kind) {
-  if (!cfg || cfg->num_blocks < 0 || cfg->num_heads <= 0) return 0;
-  return static_cast<size_t>(cfg->num_blocks) * cfg->num_heads *
+  if (!cfg || cfg->num_blocks < 0 || cfg->num_heads <= 0 || cfg->num_kv_heads < 0) return 0;
+  return static_cast<size_t>(cfg->num_blocks) * kv_heads(cfg) *
          loopkv_record_bytes(cfg->head_dim, cfg->block_size, kind);
 }
 
 size_t loopkv_residual_bytes(const loopkv_config* cfg) {
-  if (!cfg || cfg->max_batch < 0 || cfg->num_heads <= 0) return 0;
-  return static_cast<size_t>(cfg->max_batch) * cfg->num_heads * 32 * cfg->head_dim * 2;
+  if (!cfg || cfg->max_batch < 0 || cfg->num_heads <= 0 || cfg->num_kv_heads < 0) return 0;
+  return static_cast<size_t>(cfg->max_batch) * kv_heads(cfg) * 32 * cfg->head_dim * 2;
 }
 
 loopkv_status loopkv_quantize_append(const loopkv_config* cfg, const loopkv_cells* cells,
@@ -102,7 +109,7 @@ loopkv_status loopkv_quantize_append(const loopkv_config* cfg, const loopkv_cell
   p.start_pos = start_pos;
   p.err = err_flag;
   p.T = num_tokens;
-  p.H = cfg->num_heads;
+  p.H = kv_heads(cfg);
   p.max_blocks = cfg->max_blocks_per_seq;
   p.num_blocks = cfg->num_blocks;
   const cudaError_t e = loopkv::launch_append(kind, cfg->head_dim, p, batch,
@@ -117,8 +124,9 @@ int32_t loopkv_decode_splits(const loopkv_config* cfg, int32_t kind, int32_t bat
   const int cap = cfg->max_blocks_per_seq * cfg->block_size;
   const int len = max_seq_len == 0 ? cap : max_seq_len;
   if (len < 0 || len > cap || len > kMaxSeqLen) return 0;
-  if (cfg->decode_splits) return cfg->decode_splits;
-  return loopkv::decode_splits(kind, cfg->head_dim, batch, cfg->num_heads, len);
+  const int hc = loopkv::head_cluster(kind, cfg->num_heads / kv_heads(cfg), false);
+  if (cfg->decode_splits) return cfg->decode_splits <= loopkv::max_splits(hc) ? cfg->decode_splits : 0;
+  return loopkv::decode_splits(kind, cfg->head_dim, batch, cfg->num_heads, len, hc);
 }
 
 }  // extern "C"
@@ -158,10 +166,19 @@ loopkv_status decode_common(const loopkv_config* cfg, const loopkv_cells* cells,
   if (kind != LOOPKV_CELL_BF16 && (!residual || !aligned16(residual))) return LOOPKV_ERR_INVALID_ARG;
   if (!q || !aligned16(q) || !out || !block_table || !seq_lens) return LOOPKV_ERR_INVALID_ARG;
   if (fused && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return LOOPKV_ERR_INVALID_ARG;
+  const int group = cfg->num_heads / kv_heads(cfg);  // query heads per KV head
+  // grouped queries append through loopkv_quantize_append: in one launch the
+  // other heads' CTAs would read the new token before its writer is done
+  if (fused && group > 1) return LOOPKV_ERR_UNSUPPORTED;
 
+  const bool full_values = kind == LOOPKV_CELL_Q4 && tau == 0.f;
+  // splits are capped for every 4-bit source (also tau = 0) so that the
+  // choice does not depend on tau; the launch clusters heads only for tau > 0
+  const int hc = loopkv::head_cluster(kind, group, false);
+  if (cfg->decode_splits > loopkv::max_splits(hc)) return LOOPKV_ERR_UNSUPPORTED;
   const int splits = cfg->decode_splits
                          ? cfg->decode_splits
-                         : loopkv::decode_splits(kind, cfg->head_dim, batch, cfg->num_heads, len);
+                         : loopkv::decode_splits(kind, cfg->head_dim, batch, cfg->num_heads, len, hc);
   const int groups = (len + 31) / 32;
   loopkv::DecodeParams p;
   p.arena = static_cast<const uint8_t*>(arena);
@@ -174,10 +191,15 @@ loopkv_status decode_common(const loopkv_config* cfg, const loopkv_cells* cells,
   p.sel_count = sel_count;
   p.err = err_flag;
   p.H = cfg->num_heads;
+  p.Hkv = kv_heads(cfg);
+  p.g_log2 = group == 8 ? 3 : group == 4 ? 2 : group == 2 ? 1 : 0;
   p.max_blocks = cfg->max_blocks_per_seq;
   p.num_blocks = cfg->num_blocks;
   p.mask_words = (cap + 31) / 32;
   p.chunk_groups = (groups + splits - 1) / splits;
+  // one split's logits, block ids and selection words live in shared memory
+  if (loopkv::decode_smem_bytes(kind, cfg->head_dim, full_values, p.chunk_groups) > kMaxSmemPerCta)
+    return LOOPKV_ERR_UNSUPPORTED;
   p.max_seq_len = len;
   p.tau = tau;
   p.sm_scale_log2 = sm_scale * 1.4426950408889634f;
@@ -186,7 +208,6 @@ loopkv_status decode_common(const loopkv_config* cfg, const loopkv_cells* cells,
   p.v_new = static_cast<const __nv_bfloat16*>(v_new);
   p.wr_arena = fused ? static_cast<uint8_t*>(arena) : nullptr;
   p.wr_residual = fused ? static_cast<__nv_bfloat16*>(residual) : nullptr;
-  const bool full_values = kind == LOOPKV_CELL_Q4 && tau == 0.f;
   const cudaError_t e = loopkv::launch_decode(kind, cfg->head_dim, p, batch, splits, full_values,
                                               static_cast<cudaStream_t>(stream),
                                               (cfg->flags & LOOPKV_FLAG_PDL) != 0);

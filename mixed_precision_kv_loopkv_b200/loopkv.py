@@ -39,7 +39,7 @@ class loopkv_config(ctypes.Structure):
                 ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
                 ("max_batch", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32),
                 ("flags", ctypes.c_uint32), ("decode_splits", ctypes.c_int32),
-                ("plan", ctypes.POINTER(ctypes.c_uint8))]
+                ("plan", ctypes.POINTER(ctypes.c_uint8)), ("num_kv_heads", ctypes.c_int32)]
 
 
 class loopkv_cells(ctypes.Structure):
@@ -111,28 +111,32 @@ def loopkv_status_string(status: int) -> str:
 class KVCells:
     """Device storage of every (loop, layer) cell of a looped model.
 
-    Holds one arena uint8[num_blocks * H * record] per stored cell and one
-    key residual bf16[max_batch, H, 32, D] per 4-bit or 2-bit cell (torch
-    tensors), plus the C structs the entry points take.  ``allocate`` (a set
-    of cell indices) restricts storage to those cells; the others get null
-    pointers, which the entry points reject.
+    Holds one arena uint8[num_blocks * Hkv * record] per stored cell and one
+    key residual bf16[max_batch, Hkv, 32, D] per 4-bit or 2-bit cell (torch
+    tensors), plus the C structs the entry points take.  ``num_heads`` counts
+    query heads; ``num_kv_heads`` (0: as many as query heads) the KV heads
+    the cells store.  ``allocate`` (a set of cell indices) restricts storage
+    to those cells; the others get null pointers, which the entry points
+    reject.
     """
 
     def __init__(self, plan, num_loops: int, num_layers: int, num_heads: int, head_dim: int,
                  num_blocks: int, max_batch: int, max_blocks_per_seq: int, device="cuda",
-                 flags: int = 0, decode_splits: int = 0, block_size: int = 16, allocate=None):
+                 flags: int = 0, decode_splits: int = 0, block_size: int = 16, allocate=None,
+                 num_kv_heads: int = 0):
         codes = [KIND_CODES.get(k, k) for k in plan]
         if len(codes) != num_loops * num_layers:
             raise ValueError("plan must have num_loops * num_layers entries")
         self.plan_codes = codes
         self.num_loops, self.num_layers = num_loops, num_layers
         self.num_heads, self.head_dim = num_heads, head_dim
+        self.num_kv_heads = num_kv_heads or num_heads
         self.num_blocks, self.max_batch = num_blocks, max_batch
         self.max_blocks_per_seq, self.block_size = max_blocks_per_seq, block_size
         self._plan_buf = (ctypes.c_uint8 * len(codes))(*codes)
         self.cfg = loopkv_config(num_loops, num_layers, num_heads, head_dim, block_size, num_blocks,
                                  max_batch, max_blocks_per_seq, flags, decode_splits,
-                                 ctypes.cast(self._plan_buf, ctypes.POINTER(ctypes.c_uint8)))
+                                 ctypes.cast(self._plan_buf, ctypes.POINTER(ctypes.c_uint8)), num_kv_heads)
         self.arenas, self.residuals = [], []
         ptr_a = (ctypes.c_void_p * len(codes))()
         ptr_r = (ctypes.c_void_p * len(codes))()
@@ -143,7 +147,7 @@ class KVCells:
                 arena = torch.zeros(nbytes, dtype=torch.uint8, device=device)
                 ptr_a[c] = arena.data_ptr()
                 if kind in (LOOPKV_CELL_Q4, LOOPKV_CELL_Q2):
-                    residual = torch.zeros((max_batch, num_heads, 32, head_dim), dtype=torch.bfloat16,
+                    residual = torch.zeros((max_batch, self.num_kv_heads, 32, head_dim), dtype=torch.bfloat16,
                                            device=device)
                     ptr_r[c] = residual.data_ptr()
             self.arenas.append(arena)
@@ -177,14 +181,14 @@ class KVCells:
         return loopkv_record_bytes(self.head_dim, kind, self.block_size)
 
     def arena_view(self, cell: int) -> torch.Tensor:
-        """Arena of a stored cell as uint8[num_blocks, H, record]."""
+        """Arena of a stored cell as uint8[num_blocks, Hkv, record]."""
         a = self.arenas[cell]
-        return a.view(self.num_blocks, self.num_heads, -1)
+        return a.view(self.num_blocks, self.num_kv_heads, -1)
 
 
 def loopkv_quantize_append(kv: KVCells, loop: int, layer: int, k_new, v_new, block_table, start_pos,
                            err_flag=None, stream=None):
-    """Append k_new, v_new bf16[B, T, H, D] at positions start_pos[b].. (device int32)."""
+    """Append k_new, v_new bf16[B, T, Hkv, D] at positions start_pos[b].. (device int32)."""
     if k_new.dim() != 4:
         raise ValueError("k_new must be [batch, tokens, heads, head_dim]")
     batch, tokens = int(k_new.shape[0]), int(k_new.shape[1])
@@ -219,7 +223,7 @@ def loopkv_decode_attention(kv: KVCells, loop: int, layer: int, q, block_table, 
 def loopkv_append_decode_attention(kv: KVCells, loop: int, layer: int, k_new, v_new, q, block_table, start_pos,
                                    tau: float, sm_scale: float = 1.0, out=None, max_seq_len: int = 0,
                                    sel_mask=None, sel_count=None, err_flag=None, stream=None):
-    """Append token start_pos[b] (k_new, v_new bf16[B, 1, H, D]) to a stored
+    """Append token start_pos[b] (k_new, v_new bf16[B, 1, Hkv, D]) to a stored
     cell and attend q bf16[B, H, D] over start_pos[b] + 1 tokens, in one
     launch; returns out bf16[B, H, D]."""
     if out is None:

@@ -23,7 +23,7 @@ from .loopkv import (LOOPKV_CELL_REUSE, KVCells, loopkv_append_decode_attention,
 
 
 def prefill(kv: KVCells, loop: int, layer: int, k, v, block_table, lens, err_flag=None, stream=None):
-    """Append the first lens[b] tokens of k, v (bf16 [B, n_max, H, D]) to the
+    """Append the first lens[b] tokens of k, v (bf16 [B, n_max, Hkv, D]) to the
     cell, sequences of different lengths included: one append per distinct
     length, sequences already complete skipped (negative start position)."""
     lens = [int(x) for x in (lens.tolist() if hasattr(lens, "tolist") else lens)]
@@ -43,19 +43,20 @@ class LoopedDecodeStep:
 
     pos    : device int32[B], current length n of every sequence (the new
              token's position); ``advance()`` moves it by one on the device.
-    q      : per cell, bf16[B, H, D]
-    k_new, v_new : per stored cell, bf16[B, 1, H, D] (None for reuse cells)
+    q      : per cell, bf16[B, H, D]  (H query heads)
+    k_new, v_new : per stored cell, bf16[B, 1, Hkv, D] (None for reuse cells)
     out    : per cell, bf16[B, H, D] (written)
     sel_count : optional per cell int32[B, H] (written)
     fused  : a stored cell runs append and attention as one launch
-             (loopkv_append_decode_attention); False: two launches
+             (loopkv_append_decode_attention); False: two launches.  Grouped
+             queries (Hkv < H) always take two launches
     """
 
     def __init__(self, kv: KVCells, block_table, pos, q, k_new, v_new, out, tau: float,
                  sm_scale: float, max_seq_len: int, sel_count=None, err_flag=None, cells=None,
                  fused: bool = True):
         self.kv = kv
-        self.fused = fused
+        self.fused = fused and kv.num_kv_heads == kv.num_heads
         self.cells = list(range(len(kv.plan_codes))) if cells is None else sorted(cells)
         self.block_table = block_table
         self.pos = pos

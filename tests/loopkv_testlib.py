@@ -22,7 +22,7 @@ def build_store(w, cells=None, capacity=None, device="cuda", flags=0, splits=0, 
 
     ``cells`` limits which cells get storage and data (reuse cells always
     need their final-loop source).  Returns (kv, plan, table, lens, kvdata)
-    with kvdata[cell] = (K, V) bf16 [B, n_max, H, D] on the device.
+    with kvdata[cell] = (K, V) bf16 [B, n_max, Hkv, D] on the device.
     """
     from mixed_precision_kv_loopkv_b200 import KVCells, prefill as prefill_cell
 
@@ -36,7 +36,7 @@ def build_store(w, cells=None, capacity=None, device="cuda", flags=0, splits=0, 
             want.add((w.num_loops - 1) * w.num_layers + c % w.num_layers)
     kv = KVCells(plan, w.num_loops, w.num_layers, w.num_heads, w.head_dim, num_blocks,
                  w.batch, table.shape[1], device=device, flags=flags, decode_splits=splits,
-                 allocate=want)
+                 allocate=want, num_kv_heads=w.num_kv_heads)
     table_d = torch.from_numpy(table).to(device)
     lens_d = torch.from_numpy(lens).to(device)
     data = {}
@@ -59,6 +59,12 @@ def oracle_pair(kind, k, v, q, tau, sm_scale, unit=1):
     return seq.attend(q.float().cpu().numpy(), tau, sm_scale, unit)
 
 
+def oracle_group(kind, k, v, qs, tau, sm_scale, unit=1):
+    """Oracle decode of the query heads qs [G, D] sharing one KV head."""
+    seq = O.StoredSequence(kind, k.float().cpu().numpy(), v.float().cpu().numpy())
+    return seq.attend_grouped(qs.float().cpu().numpy(), tau, sm_scale, unit)
+
+
 def unpack_mask(words: torch.Tensor, n: int) -> np.ndarray:
     w = words.cpu().numpy().astype(np.int64) & 0xFFFFFFFF
     bits = ((w[:, None] >> np.arange(32)) & 1).astype(bool).reshape(-1)
@@ -67,17 +73,30 @@ def unpack_mask(words: torch.Tensor, n: int) -> np.ndarray:
 
 def check_cell(kv, plan, cell, data, q, table, lens, tau, sm_scale, pairs, out=None,
                sel_mask=None, sel_count=None, report=None, unit=1):
-    """Compare one decoded cell with the oracle on the given (b, h) pairs."""
+    """Compare one decoded cell with the oracle on the given (b, h) pairs
+    (h: query head; with grouped queries the oracle decodes every head of
+    h's KV head together, for the union of their selections)."""
     src = kv.source_cell(cell)
     kind = plan[src]
     k_all, v_all = data[src]
     lens_h = lens.cpu().numpy()
     out_h = out.float().cpu()
+    G = kv.num_heads // kv.num_kv_heads
+    groups = {}
     worst = 0.0
     mism = 0
     for (b, h) in pairs:
         n = int(lens_h[b])
-        o, sel, p = oracle_pair(kind, k_all[b, :n, h], v_all[b, :n, h], q[b, h], tau, sm_scale, unit)
+        hk = h // G
+        if G == 1:
+            o, sel, p = oracle_pair(kind, k_all[b, :n, hk], v_all[b, :n, hk], q[b, h], tau, sm_scale, unit)
+            p = p[None]
+        else:
+            if (b, hk) not in groups:
+                groups[(b, hk)] = oracle_group(kind, k_all[b, :n, hk], v_all[b, :n, hk],
+                                               q[b, hk * G:(hk + 1) * G], tau, sm_scale, unit)
+            og, sel, p = groups[(b, hk)]
+            o = og[h - hk * G]
         got = out_h[b, h].numpy().astype(np.float64)
         err = np.abs(got - o) - (ATOL + RTOL * np.abs(o))
         worst = max(worst, float(np.max(np.abs(got - o))) if n else 0.0)
@@ -88,14 +107,15 @@ def check_cell(kv, plan, cell, data, q, table, lens, tau, sm_scale, pairs, out=N
         if sel_mask is not None and n:
             g = unpack_mask(sel_mask[b, h], n)
             diff = np.nonzero(g != sel)[0]
-            # with coarser units a token follows its unit's largest weight
-            pu = p if unit == 1 else np.array([p[(t // unit) * unit: (t // unit + 1) * unit].max()
-                                               for t in range(n)])
-            bad = [t for t in diff if abs(pu[t] - tau) >= SEL_WINDOW]
+            # with coarser units a token follows its unit's largest weight;
+            # with grouped queries, the weights of every head of the group
+            pu = p if unit == 1 else np.stack([[ph[(t // unit) * unit: (t // unit + 1) * unit].max()
+                                                for t in range(n)] for ph in p])
+            bad = [t for t in diff if np.all(np.abs(pu[:, t] - tau) >= SEL_WINDOW)]
             if bad:
                 t = bad[0]
                 raise AssertionError(f"cell {cell} b={b} h={h}: token {t} selected gpu={g[t]} "
-                                     f"oracle={sel[t]} p={p[t]:.9g} tau={tau}")
+                                     f"oracle={sel[t]} p={p[:, t]} tau={tau}")
             mism += len(diff)
         if sel_count is not None:
             want = int(sel.sum())
@@ -123,3 +143,51 @@ def mask_buffers(kv, batch, device="cuda"):
     words = math.ceil(kv.max_blocks_per_seq * kv.block_size / 32)
     return (torch.zeros((batch, kv.num_heads, words), dtype=torch.int32, device=device),
             torch.zeros((batch, kv.num_heads), dtype=torch.int32, device=device))
+
+
+def step_parity(w, nseq, cells=None, extra=32, fused=True):
+    """One captured looped decode step (append + attend per cell, PDL,
+    CUDA graph) exactly as the benchmark runs it, checked on sampled
+    sequences of every cell against the oracle."""
+    from mixed_precision_kv_loopkv_b200 import LOOPKV_FLAG_PDL, LoopedDecodeStep
+    from workload import cell_new_token, seq_lens_for
+    kv, plan, table, lens, data = build_store(w, cells=cells, capacity=seq_lens_for(w) + extra,
+                                              flags=LOOPKV_FLAG_PDL)
+    run_cells = sorted(range(w.num_cells) if cells is None else
+                       set(cells) | {kv.source_cell(c) for c in cells})
+    q, kn, vn, out = {}, {}, {}, {}
+    for c in run_cells:
+        q[c] = query_for(w, c)
+        out[c] = torch.zeros_like(q[c])
+        if plan[c] != "reuse":
+            kn[c], vn[c] = cell_new_token(w, *divmod(c, w.num_layers), device="cuda")
+    pos = lens.clone()
+    max_len = int(lens.max()) + extra
+    step = LoopedDecodeStep(kv, table, pos, q, kn, vn, out, w.tau, w.sm_scale, max_len, cells=run_cells,
+                            fused=fused)
+    step.run()                      # eager warm-up; idempotent at the same position
+    torch.cuda.synchronize()
+    for c in run_cells:
+        out[c].zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step.run()
+    g.replay()
+    torch.cuda.synchronize()
+    # oracle view: stored cells hold the new token at position n
+    full = {}
+    for c, (k, v) in data.items():
+        kk = torch.cat([k, torch.zeros_like(k[:, :1])], dim=1)
+        vv = torch.cat([v, torch.zeros_like(v[:, :1])], dim=1)
+        for b in range(w.batch):
+            n = int(lens[b])
+            kk[b, n], vv[b, n] = kn[c][b, 0], vn[c][b, 0]
+        full[c] = (kk, vv)
+    pairs = sample_pairs(w, nseq)
+    report = []
+    for cell in run_cells:
+        lc = lens if plan[cell] == "reuse" else lens + 1
+        check_cell(kv, plan, cell, full, q[cell], table, lc, w.tau, w.sm_scale, pairs, out=out[cell],
+                   report=report)
+    del g
+    return report

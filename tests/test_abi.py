@@ -188,3 +188,34 @@ def test_fused_step_argument_errors(m):
 def test_two_selection_units_are_invalid(m):
     cfg = _cfg(m, [Q4], 1, 1, flags=0x2 | 0x4)
     assert _decode(m, cfg, _cells(m, 1)) == 1
+
+
+def test_grouped_query_config_checks(m):
+    """KV heads must divide the query heads, with 1, 2, 4 or 8 query heads
+    per KV head; a 4-bit source clusters G heads x splits <= 8 CTAs; the
+    fused append + decode takes no grouped queries."""
+    assert _decode(m, _cfg(m, [Q4], 1, 1, num_heads=6, num_kv_heads=4), _cells(m, 1)) == 1
+    assert _decode(m, _cfg(m, [Q4], 1, 1, num_kv_heads=-1), _cells(m, 1)) == 1
+    assert _decode(m, _cfg(m, [Q4], 1, 1, num_heads=6, num_kv_heads=2), _cells(m, 1)) == 3   # G = 3
+    assert _decode(m, _cfg(m, [Q4], 1, 1, num_heads=32, num_kv_heads=2), _cells(m, 1)) == 3  # G = 16
+    assert _append(m, _cfg(m, [Q4], 1, 1, num_heads=6, num_kv_heads=2), _cells(m, 1)) == 3
+    assert _decode(m, _cfg(m, [Q4], 1, 1, num_heads=8, num_kv_heads=2, decode_splits=4), _cells(m, 1)) == 3
+    assert _fused(m, _cfg(m, [Q4], 1, 1, num_heads=4, num_kv_heads=2), _cells(m, 1)) == 3
+
+
+def test_grouped_query_sizes_and_splits(m):
+    lib = m.library()
+    gqa = _cfg(m, [Q4], 1, 1, num_heads=8, num_kv_heads=2)
+    mha = _cfg(m, [Q4], 1, 1, num_heads=2)
+    for kind in (Q4, Q2, BF16):
+        assert lib.loopkv_arena_bytes(ctypes.byref(gqa), kind) == lib.loopkv_arena_bytes(ctypes.byref(mha), kind)
+    assert lib.loopkv_residual_bytes(ctypes.byref(gqa)) == lib.loopkv_residual_bytes(ctypes.byref(mha))
+    for g, smax in [(2, 4), (4, 2), (8, 1)]:
+        cfg = _cfg(m, [Q4], 1, 1, num_heads=2 * g, num_kv_heads=2, max_blocks_per_seq=4096)
+        for n in (256, 8192, 65536):
+            assert 1 <= lib.loopkv_decode_splits(ctypes.byref(cfg), Q4, 1, n) <= smax
+        # 2-bit sources select nothing: their splits are not capped
+        assert lib.loopkv_decode_splits(ctypes.byref(cfg), Q2, 1, 65536) == 8
+        over = _cfg(m, [Q4], 1, 1, num_heads=2 * g, num_kv_heads=2, decode_splits=2 * smax)
+        if 2 * smax <= 8:
+            assert lib.loopkv_decode_splits(ctypes.byref(over), Q4, 1, 64) == 0

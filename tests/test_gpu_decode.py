@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from loopkv_testlib import (build_store, check_cell, mask_buffers, query_for, sample_pairs)
+from loopkv_testlib import (build_store, check_cell, mask_buffers, query_for, sample_pairs, step_parity)
 from workload import block_table_for, cell_kv, get_workload
 from workload.configs import Workload
 
@@ -145,58 +145,9 @@ def test_pdl_flag_matches_plain_launch():
     assert torch.equal(a, b)
 
 
-def _step_parity(name, nseq, cells=None, extra=32, fused=True):
-    """One captured looped decode step (append + attend per cell, PDL,
-    CUDA graph) exactly as the benchmark runs it, checked on sampled
-    sequences of every cell against the oracle."""
-    from mixed_precision_kv_loopkv_b200 import LOOPKV_FLAG_PDL, LoopedDecodeStep
-    from workload import cell_new_token, seq_lens_for
-    w = get_workload(name)
-    kv, plan, table, lens, data = build_store(w, cells=cells, capacity=seq_lens_for(w) + extra,
-                                              flags=LOOPKV_FLAG_PDL)
-    run_cells = sorted(range(w.num_cells) if cells is None else
-                       set(cells) | {kv.source_cell(c) for c in cells})
-    q, kn, vn, out = {}, {}, {}, {}
-    for c in run_cells:
-        q[c] = query_for(w, c)
-        out[c] = torch.zeros_like(q[c])
-        if plan[c] != "reuse":
-            kn[c], vn[c] = cell_new_token(w, *divmod(c, w.num_layers), device="cuda")
-    pos = lens.clone()
-    max_len = int(lens.max()) + extra
-    step = LoopedDecodeStep(kv, table, pos, q, kn, vn, out, w.tau, w.sm_scale, max_len, cells=run_cells,
-                            fused=fused)
-    step.run()                      # eager warm-up; idempotent at the same position
-    torch.cuda.synchronize()
-    for c in run_cells:
-        out[c].zero_()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        step.run()
-    g.replay()
-    torch.cuda.synchronize()
-    # oracle view: stored cells hold the new token at position n
-    full = {}
-    for c, (k, v) in data.items():
-        kk = torch.cat([k, torch.zeros_like(k[:, :1])], dim=1)
-        vv = torch.cat([v, torch.zeros_like(v[:, :1])], dim=1)
-        for b in range(w.batch):
-            n = int(lens[b])
-            kk[b, n], vv[b, n] = kn[c][b, 0], vn[c][b, 0]
-        full[c] = (kk, vv)
-    pairs = sample_pairs(w, nseq)
-    report = []
-    for cell in run_cells:
-        lc = lens if plan[cell] == "reuse" else lens + 1
-        check_cell(kv, plan, cell, full, q[cell], table, lc, w.tau, w.sm_scale, pairs, out=out[cell],
-                   report=report)
-    del g
-    return report
-
-
 @pytest.mark.parametrize("fused", [True, False])
 def test_ouro_step_captured_with_pdl(fused):
-    rep = _step_parity("ouro_step", nseq=2, fused=fused)
+    rep = step_parity(get_workload("ouro_step"), nseq=2, fused=fused)
     assert len(rep) == 96
 
 
