@@ -9,8 +9,10 @@
 // softmax weight p_t >= tau.  Split-K over the context follows the
 // streaming-softmax idea (O(1)-memory attention in the same pages' listing).
 //
-// Grid (splits, heads, batch); the splits of one (sequence, head) form one
-// thread-block cluster.  Each CTA owns a chunk of 32-token groups:
+// Grid (splits, query heads, batch); the splits of one (sequence, head) form
+// one thread-block cluster (with grouped queries and a low-plane selection,
+// the splits of all query heads sharing a KV head, which OR their selections
+// into one union).  Each CTA owns a chunk of 32-token groups:
 //   - every warp streams its own groups (interleaved with the other warps)
 //     through a private ring of shared-memory stages: lane 0 issues 1-D bulk
 //     copies (TMA, no multicast) of each block record's pass-1 prefix (keys,

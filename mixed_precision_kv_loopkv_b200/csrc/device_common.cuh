@@ -2,7 +2,7 @@
 //
 // Thin inline-PTX wrappers: mbarriers, 1-D bulk copies (TMA, no multicast)
 // into the CTA's own shared memory, cluster barriers and distributed shared
-// memory loads, programmatic dependent launch, and waits bounded by the
+// memory stores, programmatic dependent launch, and waits bounded by the
 // global timer so that no kernel can spin forever.
 #pragma once
 
@@ -80,9 +80,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -129,12 +126,6 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Orders this thread's earlier generic-proxy shared-memory accesses before
-// later async-proxy (bulk copy) accesses of the same buffer.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // blockIdx.y read afresh (not merged with earlier reads, so that it need not
 // stay in a register in between)
 __device__ __forceinline__ int cta_id_y() {
@@ -144,11 +135,6 @@ __device__ __forceinline__ int cta_id_y() {
 }
 
 // ----------------------------------------------------------------- cluster
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
 // Every thread of every CTA of the cluster must call this (no early exits).
 __device__ __forceinline__ void cluster_sync_all() {
   __syncwarp();
@@ -179,16 +165,6 @@ __device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
-}
-__device__ __forceinline__ float ld_peer_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ int ld_peer_s32(uint32_t addr) {
-  int v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
 }
 
 // Stores into a peer CTA's shared memory (visible to it after the next
