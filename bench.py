@@ -26,6 +26,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -61,7 +62,27 @@ def parse_args(argv=None):
                     help="override the workload's batch (a smaller case of the same kernel)")
     ap.add_argument("--cells", type=int, default=0,
                     help="run only the first N cells (and their reuse sources): a small case for ncu")
+    ap.add_argument("--tau", type=float, default=None,
+                    help="override the workload's low-plane threshold (tau sweep; 'inf' for none)")
+    ap.add_argument("--temperature", type=float, default=None,
+                    help="override the query temperature (tau sweep: flat 0.5 .. peaky 4)")
+    ap.add_argument("--all-bf16", action="store_true",
+                    help="store every cell as bf16 (the unquantised comparison run of the tau sweep)")
     return ap.parse_args(argv)
+
+
+def apply_overrides(w, args):
+    """The workload with the command line's batch / tau / temperature / bf16 overrides."""
+    kw = {}
+    if args.batch:
+        kw["batch"] = args.batch
+    if args.tau is not None:
+        kw["tau"] = args.tau
+    if args.temperature is not None:
+        kw["temperature"] = args.temperature
+    if args.all_bf16:
+        kw["all_bf16"] = True
+    return w.with_(**kw) if kw else w
 
 
 # ----------------------------------------------------------------- ranks
@@ -357,12 +378,15 @@ def run_oracle(items, w, budget_s: float = None, steps: int = None, warmup: int 
 
 def workload_config(w, world):
     frac = f"{round(w.frac_q4 * 100)}/{round((1 - w.frac_q4 - w.frac_reuse) * 100)}/{round(w.frac_reuse * 100)}"
+    plan = "all bf16" if w.all_bf16 else f"plan {frac} 4b/2b/reuse"
     ctx = f"{w.ctx_range[0]}..{w.ctx_range[1]}" if w.ctx_range else str(w.context)
+    temp = "" if w.temperature == 1.0 else f", q temperature {w.temperature}"
     return {
         "workload": (f"{w.name}: batch {w.batch}, {w.num_loops} loops x {w.num_layers} layers, "
-                     f"{w.num_heads} MHA heads x {w.head_dim}, context {ctx}, plan {frac} "
-                     f"4b/2b/reuse, tau {w.tau}, paged 16-token blocks ({w.paging})"),
-        "batch_per_gpu": w.batch, "context": ctx, "cells": w.num_cells, "tau": w.tau,
+                     f"{w.num_heads} MHA heads x {w.head_dim}, context {ctx}, {plan}, "
+                     f"tau {w.tau}{temp}, paged 16-token blocks ({w.paging})"),
+        "batch_per_gpu": w.batch, "context": ctx, "cells": w.num_cells,
+        "tau": w.tau if math.isfinite(w.tau) else "inf", "temperature": w.temperature,
         "l2": "inputs larger than L2 (whole step streams the cache once)",
         "parallelism": f"dp{world} (sequences)",
     }
@@ -374,7 +398,7 @@ def reference_arm(args, world, rank):
     from workload import get_workload, make_plan, seq_lens_for
     if rank != 0:
         return
-    w = get_workload(args.workload)
+    w = apply_overrides(get_workload(args.workload), args)
     plan, lens = make_plan(w), seq_lens_for(w)
     items = oracle_sample(w, plan, lens, n_pairs=16)
     gbs, secs, n_run, cores = run_oracle(items, w, steps=args.steps, warmup=args.warmup)
@@ -397,9 +421,7 @@ def main_arm(args, world, rank, local):
 
     torch.cuda.set_device(local)
     init_dist(world, local)
-    w = get_workload(args.workload)
-    if args.batch:
-        w = w.with_(batch=args.batch)
+    w = apply_overrides(get_workload(args.workload), args)
     S = setup(w, pdl=not args.no_pdl, splits=args.splits, ncells=args.cells, fused=not args.no_fuse,
               unit=args.select_unit)
     step, plan, lens = S["step"], S["plan"], S["lens"]

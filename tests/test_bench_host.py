@@ -67,3 +67,20 @@ def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("demo") == 1234.0
     (csrc / "decode.cu").write_text("// changed\n")
     assert bench.profiled_traffic("demo") is None
+
+
+def test_sweep_overrides_and_strict_json():
+    """The tau sweep's overrides reach the workload, and the config stays
+    strict JSON for tau = +inf."""
+    import json
+    import math
+    from workload import get_workload
+    args = bench.parse_args(["--workload", "tau_sweep", "--tau", "inf", "--temperature", "4", "--all-bf16",
+                             "--batch", "2"])
+    w = bench.apply_overrides(get_workload(args.workload), args)
+    assert math.isinf(w.tau) and w.temperature == 4.0 and w.all_bf16 and w.batch == 2
+    cfg = bench.workload_config(w, 1)
+    text = json.dumps(cfg, allow_nan=False)
+    assert '"tau": "inf"' in text and "all bf16" in cfg["workload"] and "temperature 4.0" in cfg["workload"]
+    plain = bench.apply_overrides(get_workload("ouro_step"), bench.parse_args([]))
+    assert plain == get_workload("ouro_step")
