@@ -219,3 +219,13 @@ def test_grouped_query_sizes_and_splits(m):
         over = _cfg(m, [Q4], 1, 1, num_heads=2 * g, num_kv_heads=2, decode_splits=2 * smax)
         if 2 * smax <= 8:
             assert lib.loopkv_decode_splits(ctypes.byref(over), Q4, 1, 64) == 0
+
+
+def test_grouped_query_context_beyond_one_cta_is_unsupported(m):
+    """Eight query heads per KV head leave one split per cluster: a 64K
+    context would not fit one CTA's shared memory, 16K does (no launch
+    here: the 16K call fails only later, at the fake pointers' launch)."""
+    big = _cfg(m, [Q4], 1, 1, num_heads=16, num_kv_heads=2, max_blocks_per_seq=4096)
+    assert _decode(m, big, _cells(m, 1), max_seq_len=65536) == 3
+    lib = m.library()
+    assert lib.loopkv_decode_splits(ctypes.byref(big), Q4, 1, 16384) == 1
