@@ -277,6 +277,65 @@ def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0, fused: bo
                 out_all=out_all, sel_all=sel_all)
 
 
+def time_end_to_end(g, S, steps):
+    """Device time (ms) of ``steps`` steps fed from and drained to pinned
+    host memory: every step copies its queries and new tokens in from the
+    host and its outputs back out.  The copies run on a second stream
+    through two sets of staging buffers, one step ahead of (inputs) and one
+    behind (outputs) the step's kernels, so transfers overlap computation;
+    the step itself only adds two device-to-device copies.  The timed region
+    spans the first host-to-device copy to the last device-to-host copy.
+    Returns (ms, host-to-device bytes per step, device-to-host bytes per step)."""
+    ins = [S["q_all"], S["kn_all"], S["vn_all"]]
+    out = S["out_all"]
+    host_in = [t.cpu().pin_memory() for t in ins]
+    host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    stage_in = [[torch.empty_like(t) for t in ins] for _ in range(2)]
+    stage_out = [torch.empty_like(out) for _ in range(2)]
+    comp, copy = torch.cuda.current_stream(), torch.cuda.Stream()
+    in_ready, in_free, out_ready, out_free = ([torch.cuda.Event() for _ in range(2)] for _ in range(4))
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    for e in in_free + out_free:
+        e.record(comp)
+    copy.wait_stream(comp)
+
+    def h2d(i):
+        k = i % 2
+        with torch.cuda.stream(copy):
+            copy.wait_event(in_free[k])
+            for st, h in zip(stage_in[k], host_in):
+                st.copy_(h, non_blocking=True)
+            in_ready[k].record(copy)
+
+    h2d(0)
+    for i in range(steps):
+        k = i % 2
+        if i + 1 < steps:
+            h2d(i + 1)
+        comp.wait_event(in_ready[k])
+        for t, st in zip(ins, stage_in[k]):
+            t.copy_(st, non_blocking=True)
+        in_free[k].record(comp)
+        g.replay()
+        comp.wait_event(out_free[k])
+        stage_out[k].copy_(out, non_blocking=True)
+        out_ready[k].record(comp)
+        with torch.cuda.stream(copy):
+            copy.wait_event(out_ready[k])
+            host_out[k].copy_(stage_out[k], non_blocking=True)
+            out_free[k].record(copy)
+    comp.wait_stream(copy)
+    b.record(comp)
+    b.synchronize()
+    if not torch.equal(host_out[(steps - 1) % 2], out.cpu()):
+        raise RuntimeError("end-to-end outputs differ from the device result")
+    h2d_bytes = sum(h.numel() * h.element_size() for h in host_in)
+    d2h_bytes = out.numel() * out.element_size()
+    return a.elapsed_time(b), h2d_bytes, d2h_bytes
+
+
 class DecodeOnly:
     """The decode launches of a step without the appends (roofline timing)."""
 
@@ -459,26 +518,10 @@ def main_arm(args, world, rank, local):
 
     # end to end: inputs of every step copied in from pinned host memory,
     # outputs copied back, inside the timed region
-    q_h = S["q_all"].cpu().pin_memory()
-    kn_h = S["kn_all"].cpu().pin_memory()
-    vn_h = S["vn_all"].cpu().pin_memory()
-    out_h = torch.empty(S["out_all"].shape, dtype=S["out_all"].dtype).pin_memory()
     e2e_steps = max(3, args.steps // 4)
     barrier(world)
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(e2e_steps):
-        S["q_all"].copy_(q_h, non_blocking=True)
-        S["kn_all"].copy_(kn_h, non_blocking=True)
-        S["vn_all"].copy_(vn_h, non_blocking=True)
-        g.replay()
-        out_h.copy_(S["out_all"], non_blocking=True)
-    b.record()
-    b.synchronize()
-    e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
-    h2d = q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2
-    d2h = out_h.numel() * 2
+    e2e_ms, h2d, d2h = time_end_to_end(g, S, e2e_steps)
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     e2e_value = aggregate_value(bytes_step * e2e_steps, world, e2e_ms / 1e3)
 
     cpu = None
