@@ -1037,8 +1037,11 @@ long resident_ctas_t(int cg, int splits, int hc, int sms) {
   return static_cast<long>(clusters) * splits * hc;
 }
 
+// balance: ask the hardware to place a cluster's CTAs on the least loaded
+// SMs (cluster scheduling policy "load balancing") instead of the default.
 template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB, bool GQ>
-cudaError_t launch_t(const DecodeParams& p, int batch, int splits, int hc, cudaStream_t stream, bool pdl) {
+cudaError_t launch_t(const DecodeParams& p, int batch, int splits, int hc, cudaStream_t stream, bool pdl,
+                     bool balance) {
   const size_t smem = smem_bytes_t<KIND, D, FULLV>(p.chunk_groups);
   if (smem > 227u * 1024u) return cudaErrorInvalidValue;
   auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>;
@@ -1049,7 +1052,7 @@ cudaError_t launch_t(const DecodeParams& p, int batch, int splits, int hc, cudaS
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   int na = 0;
   if (CLUSTER) {
     attr[na].id = cudaLaunchAttributeClusterDimension;
@@ -1057,6 +1060,11 @@ cudaError_t launch_t(const DecodeParams& p, int batch, int splits, int hc, cudaS
     attr[na].val.clusterDim.y = hc;
     attr[na].val.clusterDim.z = 1;
     ++na;
+    if (balance) {
+      attr[na].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+      attr[na].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicyLoadBalancing;
+      ++na;
+    }
   }
   if (pdl) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1078,6 +1086,12 @@ long resident_m(int cg, int splits, int hc, int sms) {
 // 5-per-SM build: its extra warps hide latency once every SM stays busy for
 // long; short grids keep the full register budget.
 constexpr long kHighOccupancyWaves = 3;
+// Grids of at most this many waves let the hardware load-balance each
+// cluster's CTAs over the SMs: a short grid cannot spread evenly (512 CTAs
+// on 148 SMs leave some SMs one CTA more), and the busiest SMs set the
+// launch time; longer grids keep the default placement, which measured
+// faster there.
+constexpr long kBalancedWaves = 2;
 
 template <int KIND, int D, bool FULLV>
 cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
@@ -1086,20 +1100,21 @@ cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t 
   const int hc = head_cluster(KIND, 1 << p.g_log2, FULLV);
   if (splits * hc > 8) return cudaErrorInvalidValue;
   const bool cl = splits * hc > 1;
+  const long ctas = static_cast<long>(batch) * p.H * splits;
+  const long slots4 = resident_m<KIND, D, FULLV, 4>(p.chunk_groups, splits, hc, sms);
+  const bool balance = cl && slots4 > 0 && ctas <= kBalancedWaves * slots4;
   // grouped queries: one build, at four CTAs per SM
   if (p.g_log2 > 0)
-    return cl ? launch_t<KIND, D, FULLV, true, 4, true>(p, batch, splits, hc, stream, pdl)
-              : launch_t<KIND, D, FULLV, false, 4, true>(p, batch, splits, 1, stream, pdl);
+    return cl ? launch_t<KIND, D, FULLV, true, 4, true>(p, batch, splits, hc, stream, pdl, balance)
+              : launch_t<KIND, D, FULLV, false, 4, true>(p, batch, splits, 1, stream, pdl, false);
   if constexpr (KIND != LOOPKV_CELL_BF16 && !FULLV) {
-    const long ctas = static_cast<long>(batch) * p.H * splits;
-    const long slots4 = resident_m<KIND, D, FULLV, 4>(p.chunk_groups, splits, 1, sms);
     if (slots4 > 0 && ctas >= kHighOccupancyWaves * slots4 &&
         resident_m<KIND, D, FULLV, 5>(p.chunk_groups, splits, 1, sms) > slots4)
-      return cl ? launch_t<KIND, D, FULLV, true, 5, false>(p, batch, splits, 1, stream, pdl)
-                : launch_t<KIND, D, FULLV, false, 5, false>(p, batch, splits, 1, stream, pdl);
+      return cl ? launch_t<KIND, D, FULLV, true, 5, false>(p, batch, splits, 1, stream, pdl, balance)
+                : launch_t<KIND, D, FULLV, false, 5, false>(p, batch, splits, 1, stream, pdl, false);
   }
-  return cl ? launch_t<KIND, D, FULLV, true, 4, false>(p, batch, splits, 1, stream, pdl)
-            : launch_t<KIND, D, FULLV, false, 4, false>(p, batch, splits, 1, stream, pdl);
+  return cl ? launch_t<KIND, D, FULLV, true, 4, false>(p, batch, splits, 1, stream, pdl, balance)
+            : launch_t<KIND, D, FULLV, false, 4, false>(p, batch, splits, 1, stream, pdl, false);
 }
 
 // Co-resident CTAs of one decode build (0 without a device); minb 5 only
