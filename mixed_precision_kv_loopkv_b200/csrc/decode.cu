@@ -546,7 +546,10 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   // rank split + S * (h % G), so that the heads can merge their selections.
   constexpr bool head_cl = GQ && CLUSTER && C::kLogits;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_allow_dependents();
+  // Long grids let the next kernel launch at once; a grid of one wave lets
+  // it launch only after its pass 1, so that the next kernel's first CTAs
+  // do not stream into the spare slots while this one is still streaming.
+  if (p.pdl_early) pdl_allow_dependents();
   // Speculative block ids: the first 16 iterations' table entries of batch
   // slot z, for the chunk this split would get from a sequence of the host
   // bound max_seq_len.  They are used below when the actual sequence and
@@ -714,6 +717,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     }
   }
   pdl_wait_prior_grid();  // nothing below may run ahead of the previous kernel
+  if (!p.pdl_early) pdl_allow_dependents();
 
   // ---- this warp's result in its own scale 2^-m_w: true per-channel sums,
   //      reduced over the token sub-groups
@@ -1103,18 +1107,20 @@ cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t 
   const long ctas = static_cast<long>(batch) * p.H * splits;
   const long slots4 = resident_m<KIND, D, FULLV, 4>(p.chunk_groups, splits, hc, sms);
   const bool balance = cl && slots4 > 0 && ctas <= kBalancedWaves * slots4;
+  DecodeParams q = p;
+  q.pdl_early = slots4 <= 0 || ctas > slots4;
   // grouped queries: one build, at four CTAs per SM
   if (p.g_log2 > 0)
-    return cl ? launch_t<KIND, D, FULLV, true, 4, true>(p, batch, splits, hc, stream, pdl, balance)
-              : launch_t<KIND, D, FULLV, false, 4, true>(p, batch, splits, 1, stream, pdl, false);
+    return cl ? launch_t<KIND, D, FULLV, true, 4, true>(q, batch, splits, hc, stream, pdl, balance)
+              : launch_t<KIND, D, FULLV, false, 4, true>(q, batch, splits, 1, stream, pdl, false);
   if constexpr (KIND != LOOPKV_CELL_BF16 && !FULLV) {
     if (slots4 > 0 && ctas >= kHighOccupancyWaves * slots4 &&
         resident_m<KIND, D, FULLV, 5>(p.chunk_groups, splits, 1, sms) > slots4)
-      return cl ? launch_t<KIND, D, FULLV, true, 5, false>(p, batch, splits, 1, stream, pdl, balance)
-                : launch_t<KIND, D, FULLV, false, 5, false>(p, batch, splits, 1, stream, pdl, false);
+      return cl ? launch_t<KIND, D, FULLV, true, 5, false>(q, batch, splits, 1, stream, pdl, balance)
+                : launch_t<KIND, D, FULLV, false, 5, false>(q, batch, splits, 1, stream, pdl, false);
   }
-  return cl ? launch_t<KIND, D, FULLV, true, 4, false>(p, batch, splits, 1, stream, pdl, balance)
-            : launch_t<KIND, D, FULLV, false, 4, false>(p, batch, splits, 1, stream, pdl, false);
+  return cl ? launch_t<KIND, D, FULLV, true, 4, false>(q, batch, splits, 1, stream, pdl, balance)
+            : launch_t<KIND, D, FULLV, false, 4, false>(q, batch, splits, 1, stream, pdl, false);
 }
 
 // Co-resident CTAs of one decode build (0 without a device); minb 5 only

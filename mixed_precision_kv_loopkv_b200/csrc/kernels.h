@@ -37,6 +37,7 @@ struct DecodeParams {              // H = query heads, Hkv = KV heads
   float tau;
   float sm_scale_log2;            // sm_scale * log2(e)
   int sel_unit;                   // low-plane selection unit: 1, 16 or 32 tokens
+  int pdl_early;                  // set by the launcher: signal dependents at kernel start (else after pass 1)
   // fused append (k_new non-null): seq_lens holds start positions; the
   // kernel first stores token start_pos[b] into the cell, then attends over
   // start_pos[b] + 1 tokens (negative start: sequence skipped)
