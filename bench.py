@@ -68,6 +68,8 @@ def parse_args(argv=None):
                     help="override the query temperature (tau sweep: flat 0.5 .. peaky 4)")
     ap.add_argument("--all-bf16", action="store_true",
                     help="store every cell as bf16 (the unquantised comparison run of the tau sweep)")
+    ap.add_argument("--kv-heads", type=int, default=0,
+                    help="KV heads (grouped queries: the workload's query heads share them; 0 = one per head)")
     return ap.parse_args(argv)
 
 
@@ -82,6 +84,8 @@ def apply_overrides(w, args):
         kw["temperature"] = args.temperature
     if args.all_bf16:
         kw["all_bf16"] = True
+    if args.kv_heads:
+        kw["num_kv_heads"] = args.kv_heads
     return w.with_(**kw) if kw else w
 
 
@@ -242,7 +246,7 @@ def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0, fused: bo
         src = lambda c: c if plan[c] != "reuse" else (w.num_loops - 1) * w.num_layers + c % w.num_layers
         run = sorted(set(range(ncells)) | {src(c) for c in range(ncells)})
     kv = KVCells(plan, w.num_loops, w.num_layers, w.num_heads, w.head_dim, num_blocks, w.batch,
-                 table_np.shape[1],
+                 table_np.shape[1], num_kv_heads=w.num_kv_heads,
                  flags=(LOOPKV_FLAG_PDL if pdl else 0) | {1: 0, 16: LOOPKV_FLAG_SELECT_BLOCK,
                                                           32: LOOPKV_FLAG_SELECT_GROUP}[unit],
                  decode_splits=splits,
@@ -258,7 +262,7 @@ def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0, fused: bo
     if int(err):
         raise RuntimeError(f"prefill flagged device error {int(err)}")
     q_all = torch.stack([cell_query(w, *divmod(c, w.num_layers), device="cuda") for c in range(C)])
-    kn_all = torch.empty((len(stored), w.batch, 1, w.num_heads, w.head_dim), dtype=torch.bfloat16,
+    kn_all = torch.empty((len(stored), w.batch, 1, w.kv_heads, w.head_dim), dtype=torch.bfloat16,
                          device="cuda")
     vn_all = torch.empty_like(kn_all)
     for i, c in enumerate(stored):
@@ -387,19 +391,29 @@ def oracle_sample(w, plan, lens, n_pairs: int, seed: int = 0):
     for cell in cells:
         cell = int(cell)
         src = cell if plan[cell] != "reuse" else (w.num_loops - 1) * w.num_layers + cell % w.num_layers
-        b, h = int(rng.integers(w.batch)), int(rng.integers(w.num_heads))
+        g = w.num_heads // w.kv_heads
+        b, hk = int(rng.integers(w.batch)), int(rng.integers(w.kv_heads))
         n = int(lens[b])
         # the GPU arm's inputs come from the CUDA generator; without a GPU the
         # CPU generator gives inputs of the same distribution
         dev = "cuda" if torch.cuda.is_available() else "cpu"
         k, v = cell_kv(w, *divmod(src, w.num_layers), device=dev)
-        kk = k[b, :n, h].float().cpu().numpy()
-        vv = v[b, :n, h].float().cpu().numpy()
+        kk = k[b, :n, hk].float().cpu().numpy()
+        vv = v[b, :n, hk].float().cpu().numpy()
         del k, v
-        q = cell_query(w, *divmod(cell, w.num_layers), device=dev)[b, h].float().cpu().numpy()
+        # the query heads of KV head hk (one head without grouped queries)
+        q = cell_query(w, *divmod(cell, w.num_layers), device=dev)[b, hk * g:(hk + 1) * g].float().cpu().numpy()
         items.append((plan[src], O.StoredSequence(plan[src], kk, vv), q, n))
     torch.cuda.empty_cache()
     return items
+
+
+def oracle_decode(seq, q, w):
+    """The oracle's decode of one sampled item: q [G, D] holds the query heads
+    of one KV head (G = 1 without grouped queries).  Returns the selection."""
+    if len(q) == 1:
+        return seq.attend(q[0], w.tau, w.sm_scale)[1]
+    return seq.attend_grouped(q, w.tau, w.sm_scale)[1]
 
 
 def run_oracle(items, w, budget_s: float = None, steps: int = None, warmup: int = 0):
@@ -414,13 +428,13 @@ def run_oracle(items, w, budget_s: float = None, steps: int = None, warmup: int 
         try:
             for i in range(warmup):
                 kind, seq, q, n = items[i % len(items)]
-                seq.attend(q, w.tau, w.sm_scale)
+                oracle_decode(seq, q, w)
             t0 = time.perf_counter()
             i = 0
             while True:
                 kind, seq, q, n = items[i % len(items)]
-                o, sel, _ = seq.attend(q, w.tau, w.sm_scale)
-                total_bytes += decode_bytes(kind, w.head_dim, n, int(sel.sum()))
+                sel = oracle_decode(seq, q, w)
+                total_bytes += decode_bytes(kind, w.head_dim, n, int(sel.sum())) + (len(q) - 1) * 4 * w.head_dim
                 i += 1
                 el = time.perf_counter() - t0
                 if steps is not None and i >= steps:
@@ -440,9 +454,11 @@ def workload_config(w, world):
     plan = "all bf16" if w.all_bf16 else f"plan {frac} 4b/2b/reuse"
     ctx = f"{w.ctx_range[0]}..{w.ctx_range[1]}" if w.ctx_range else str(w.context)
     temp = "" if w.temperature == 1.0 else f", q temperature {w.temperature}"
+    heads = (f"{w.num_heads} MHA heads" if w.kv_heads == w.num_heads
+             else f"{w.num_heads} query heads on {w.kv_heads} KV heads")
     return {
         "workload": (f"{w.name}: batch {w.batch}, {w.num_loops} loops x {w.num_layers} layers, "
-                     f"{w.num_heads} MHA heads x {w.head_dim}, context {ctx}, {plan}, "
+                     f"{heads} x {w.head_dim}, context {ctx}, {plan}, "
                      f"tau {w.tau}{temp}, paged 16-token blocks ({w.paging})"),
         "batch_per_gpu": w.batch, "context": ctx, "cells": w.num_cells,
         "tau": w.tau if math.isfinite(w.tau) else "inf", "temperature": w.temperature,
@@ -498,6 +514,7 @@ def main_arm(args, world, rank, local):
 
     sel = S["sel_all"].cpu().numpy()
     bytes_step = step_bytes(plan, w.num_layers, w.num_loops, w.head_dim, w.num_heads, lens + 1, lens, sel,
+                            group=w.num_heads // w.kv_heads,
                             cells=step.cells)
     value = aggregate_value(bytes_step * args.steps, world, ms_max / 1e3)
     us_step = ms_max / args.steps * 1e3
@@ -510,9 +527,14 @@ def main_arm(args, world, rank, local):
     per_launch_s = ms_dec / 1e3 / (reps * launches)
     achieved = bytes_step / launches / per_launch_s / 1e9
     peak, peak_kind = hbm_peak()
-    traffic = profiled_traffic(w.name)
+    # the committed ncu counters describe the workload as defined; any
+    # override of its shape or launch options leaves them unused
+    as_profiled = not (args.batch or args.cells or args.splits or args.kv_heads or args.all_bf16 or args.no_fuse
+                       or args.no_pdl or args.select_unit != 1 or args.tau is not None
+                       or args.temperature is not None)
+    traffic = profiled_traffic(w.name) if as_profiled else None
     try:
-        inst_per_launch = float(profiled_fields(w.name)["warp_instructions_per_launch"])
+        inst_per_launch = float(profiled_fields(w.name)["warp_instructions_per_launch"]) if as_profiled else None
     except (KeyError, ValueError):
         inst_per_launch = None
 
@@ -528,8 +550,9 @@ def main_arm(args, world, rank, local):
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         items = oracle_sample(w, plan, lens, n_pairs=12)
         gbs, secs, n_run, cores = run_oracle(items, w, budget_s=args.cpu_seconds, warmup=2)
+        unit = "head" if w.kv_heads == w.num_heads else f"KV head with its {w.num_heads // w.kv_heads} query heads"
         cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n_run} (cell, sequence, head) decodes over {secs:.1f} s, round robin over "
+               "sample": f"{n_run} (cell, sequence, {unit}) decodes over {secs:.1f} s, round robin over "
                          f"12 seeded pairs of the {w.name} workload (numpy fp64, one BLAS thread)"}
 
     if rank == 0:

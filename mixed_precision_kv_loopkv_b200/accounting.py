@@ -38,10 +38,15 @@ def decode_bytes(kind: str, d: int, n: int, n_selected: int = 0) -> int:
 
 
 def step_bytes(plan, num_layers: int, num_loops: int, d: int, heads: int, lens_stored, lens_reuse,
-               selected=None, cells=None) -> int:
+               selected=None, cells=None, group: int = 1) -> int:
     """Bytes of one looped decode step: every cell decodes every (sequence,
     head); stored cells over lens_stored[b] tokens, reuse cells over the
-    final loop's lens_reuse[b]; selected[cell][b][h] low-plane rows."""
+    final loop's lens_reuse[b]; selected[cell][b][h] low-plane rows.
+
+    ``group`` query heads share one KV head (``heads`` counts query heads):
+    the KV head's cache, and the low-plane rows of the union of the group's
+    selections (reported identically for every head of the group), are
+    counted once per group; queries and outputs once per query head."""
     total = 0
     for cell, kind in enumerate(plan):
         if cells is not None and cell not in cells:
@@ -50,7 +55,7 @@ def step_bytes(plan, num_layers: int, num_loops: int, d: int, heads: int, lens_s
         src_kind = plan[src]
         lens = lens_reuse if kind == "reuse" else lens_stored
         for b, n in enumerate(lens):
-            for h in range(heads):
-                sel = 0 if selected is None else int(selected[cell][b][h])
-                total += decode_bytes(src_kind, d, int(n), sel)
+            for hk in range(heads // group):
+                sel = 0 if selected is None else int(selected[cell][b][hk * group])
+                total += decode_bytes(src_kind, d, int(n), sel) + (group - 1) * 2 * d * 2
     return total

@@ -26,3 +26,21 @@ def test_step_bytes_resolves_reuse():
     b1 = step_bytes(plan, 2, 2, 128, 1, [64], [64])
     want = 2 * decode_bytes("q4", 128, 64) + decode_bytes("q2", 128, 64) + decode_bytes("q4", 128, 64)
     assert b1 == want
+
+
+def test_grouped_queries_count_the_cache_once_per_group():
+    """G query heads on one KV head: the cache and the union's low-plane rows
+    once per KV head, queries and outputs once per query head."""
+    from mixed_precision_kv_loopkv_b200.accounting import decode_bytes, step_bytes
+    plan, lens = ["q4", "q2"], [100, 33]
+    sel = [[[5, 5, 5, 5, 7, 7, 7, 7]] * 2, [[0] * 8] * 2]
+    got = step_bytes(plan, 2, 1, 128, 8, lens, lens, sel, group=4)
+    want = 0
+    for b, n in enumerate(lens):
+        for s4 in (5, 7):
+            want += decode_bytes("q4", 128, n, s4) + 3 * 2 * 128 * 2
+        want += 2 * (decode_bytes("q2", 128, n) + 3 * 2 * 128 * 2)
+    assert got == want
+    # one query per KV head: the per-head sum
+    assert step_bytes(plan, 2, 1, 128, 2, lens, lens, [[[5, 7]] * 2, [[0, 0]] * 2]) == sum(
+        decode_bytes(k, 128, n, s) for k, ss in (("q4", (5, 7)), ("q2", (0, 0))) for n in lens for s in ss)
