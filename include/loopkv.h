@@ -196,7 +196,7 @@ LOOPKV_API loopkv_status loopkv_quantize_append(const loopkv_config* cfg, const 
  *   err_flag    : optional device int32
  * Errors: INVALID_ARG for tau < 0 or NaN, null required pointers, batch
  * outside [0, max_batch]; BAD_PLAN; UNSUPPORTED for max_seq_len above 65536,
- * for a 4-bit source with G x decode_splits above 8 (the CTAs of one KV
+ * for a 4-bit source with G x decode_splits above 16 (the CTAs of one KV
  * head's query heads and splits form one thread-block cluster), or for a
  * context split too long for one CTA's shared memory.
  */

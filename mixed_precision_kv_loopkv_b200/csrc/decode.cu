@@ -542,7 +542,8 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   const int hk = GQ ? static_cast<int>(blockIdx.y) >> p.g_log2 : static_cast<int>(blockIdx.y);
   const int Hkv = GQ ? p.Hkv : p.H;
   // Grouped queries with a low-plane selection: the CTAs of the G query
-  // heads of one KV head (and all their splits) form one cluster of S x G,
+  // heads of one KV head (and all their splits) form one cluster of S x G
+  // (up to 16 CTAs),
   // rank split + S * (h % G), so that the heads can merge their selections.
   constexpr bool head_cl = GQ && CLUSTER && C::kLogits;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1020,6 +1021,9 @@ long resident_ctas_t(int cg, int splits, int hc, int sms) {
   auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return 0;
+  if (CLUSTER && splits * hc > 8 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    return 0;
   if (!CLUSTER) {
     int blocks = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kThreads, smem) != cudaSuccess) return 0;
@@ -1051,6 +1055,10 @@ cudaError_t launch_t(const DecodeParams& p, int batch, int splits, int hc, cudaS
   auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  if (CLUSTER && splits * hc > 8) {  // grouped queries: up to 16 CTAs per cluster
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(splits, p.H, batch);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1102,7 +1110,7 @@ cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t 
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int hc = head_cluster(KIND, 1 << p.g_log2, FULLV);
-  if (splits * hc > 8) return cudaErrorInvalidValue;
+  if (splits > kMaxClusterSplits || splits * hc > kMaxClusterCtas) return cudaErrorInvalidValue;
   const bool cl = splits * hc > 1;
   const long ctas = static_cast<long>(batch) * p.H * splits;
   const long slots4 = resident_m<KIND, D, FULLV, 4>(p.chunk_groups, splits, hc, sms);

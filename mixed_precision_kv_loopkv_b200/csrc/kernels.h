@@ -56,11 +56,16 @@ inline int head_cluster(int kind, int group, bool full_values) {
   return (kind == LOOPKV_CELL_Q4 && !full_values && group > 1) ? group : 1;
 }
 
+// Largest cluster: the portable size of 8 CTAs for splits alone, 16 (a
+// non-portable size B200 supports) for splits x heads of grouped queries.
+constexpr int kMaxClusterSplits = 8;
+constexpr int kMaxClusterCtas = 16;
+
 // Largest split count (a power of two) whose cluster of splits x hc CTAs
-// stays within the portable cluster size of 8.
+// stays within kMaxClusterCtas.
 inline int max_splits(int hc) {
   int s = 1;
-  while (s < 8 && 2 * s * hc <= 8) s <<= 1;
+  while (s < kMaxClusterSplits && 2 * s * hc <= kMaxClusterCtas) s <<= 1;
   return s;
 }
 

@@ -192,14 +192,14 @@ def test_two_selection_units_are_invalid(m):
 
 def test_grouped_query_config_checks(m):
     """KV heads must divide the query heads, with 1, 2, 4 or 8 query heads
-    per KV head; a 4-bit source clusters G heads x splits <= 8 CTAs; the
+    per KV head; a 4-bit source clusters G heads x splits <= 16 CTAs; the
     fused append + decode takes no grouped queries."""
     assert _decode(m, _cfg(m, [Q4], 1, 1, num_heads=6, num_kv_heads=4), _cells(m, 1)) == 1
     assert _decode(m, _cfg(m, [Q4], 1, 1, num_kv_heads=-1), _cells(m, 1)) == 1
     assert _decode(m, _cfg(m, [Q4], 1, 1, num_heads=6, num_kv_heads=2), _cells(m, 1)) == 3   # G = 3
     assert _decode(m, _cfg(m, [Q4], 1, 1, num_heads=32, num_kv_heads=2), _cells(m, 1)) == 3  # G = 16
     assert _append(m, _cfg(m, [Q4], 1, 1, num_heads=6, num_kv_heads=2), _cells(m, 1)) == 3
-    assert _decode(m, _cfg(m, [Q4], 1, 1, num_heads=8, num_kv_heads=2, decode_splits=4), _cells(m, 1)) == 3
+    assert _decode(m, _cfg(m, [Q4], 1, 1, num_heads=8, num_kv_heads=2, decode_splits=8), _cells(m, 1)) == 3
     assert _fused(m, _cfg(m, [Q4], 1, 1, num_heads=4, num_kv_heads=2), _cells(m, 1)) == 3
 
 
@@ -210,7 +210,7 @@ def test_grouped_query_sizes_and_splits(m):
     for kind in (Q4, Q2, BF16):
         assert lib.loopkv_arena_bytes(ctypes.byref(gqa), kind) == lib.loopkv_arena_bytes(ctypes.byref(mha), kind)
     assert lib.loopkv_residual_bytes(ctypes.byref(gqa)) == lib.loopkv_residual_bytes(ctypes.byref(mha))
-    for g, smax in [(2, 4), (4, 2), (8, 1)]:
+    for g, smax in [(2, 8), (4, 4), (8, 2)]:
         cfg = _cfg(m, [Q4], 1, 1, num_heads=2 * g, num_kv_heads=2, max_blocks_per_seq=4096)
         for n in (256, 8192, 65536):
             assert 1 <= lib.loopkv_decode_splits(ctypes.byref(cfg), Q4, 1, n) <= smax
@@ -221,11 +221,9 @@ def test_grouped_query_sizes_and_splits(m):
             assert lib.loopkv_decode_splits(ctypes.byref(over), Q4, 1, 64) == 0
 
 
-def test_grouped_query_context_beyond_one_cta_is_unsupported(m):
-    """Eight query heads per KV head leave one split per cluster: a 64K
-    context would not fit one CTA's shared memory, 16K does (no launch
-    here: the 16K call fails only later, at the fake pointers' launch)."""
+def test_grouped_query_split_cap(m):
+    """Eight query heads per KV head leave two splits per cluster of 16."""
     big = _cfg(m, [Q4], 1, 1, num_heads=16, num_kv_heads=2, max_blocks_per_seq=4096)
-    assert _decode(m, big, _cells(m, 1), max_seq_len=65536) == 3
     lib = m.library()
-    assert lib.loopkv_decode_splits(ctypes.byref(big), Q4, 1, 16384) == 1
+    assert lib.loopkv_decode_splits(ctypes.byref(big), Q4, 1, 16384) == 2
+    assert lib.loopkv_decode_splits(ctypes.byref(big), Q4, 1, 65536) == 2

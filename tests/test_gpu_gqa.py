@@ -95,9 +95,9 @@ def test_grouped_selection_units(unit):
     assert int(sc.sum()) > 0
 
 
-@pytest.mark.parametrize("g,splits", [(2, 1), (2, 2), (2, 4), (4, 1), (4, 2), (8, 1)])
+@pytest.mark.parametrize("g,splits", [(2, 1), (2, 2), (2, 4), (2, 8), (4, 1), (4, 2), (4, 4), (8, 1), (8, 2)])
 def test_grouped_explicit_splits(g, splits):
-    """Every cluster shape of splits x heads up to 8 CTAs."""
+    """Every cluster shape of splits x heads up to 16 CTAs."""
     w, kv, data, table, lens = _store("q4", 128, [7, 255, 777, 3000], 2 * g, 2, seed=44, splits=splits)
     q = query_for(w, 0, temperature=4.0)
     out, sm, sc = _decode(kv, q, table, lens, 0.01)
@@ -126,13 +126,13 @@ def test_identical_queries_match_one_query_per_head():
     assert int(sc.sum()) > 0
 
 
-def test_grouped_long_context_one_split():
-    """Eight heads per KV head leave one split per cluster: a 16K-token
-    context is one CTA's chunk of 512 groups."""
+def test_grouped_long_context_two_splits():
+    """Eight heads per KV head leave two splits per cluster of 16 CTAs: a
+    16K-token context is two chunks of 256 groups."""
     from mixed_precision_kv_loopkv_b200 import loopkv_decode_splits
     lens = [16384, 9000]
     w, kv, data, table, lens_d = _store("q4", 128, lens, 16, 2, seed=46)
-    assert loopkv_decode_splits(kv, "q4", 2, 16384) == 1
+    assert loopkv_decode_splits(kv, "q4", 2, 16384) == 2
     q = query_for(w, 0, temperature=6.0)
     out, sm, sc = _decode(kv, q, table, lens_d, 0.01)
     check_cell(kv, ["q4"], 0, data, q, table, lens_d, 0.01, 1.0, [(b, h) for b in range(2) for h in (0, 7, 8, 15)],
