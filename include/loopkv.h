@@ -266,6 +266,17 @@ LOOPKV_API loopkv_status loopkv_plan_cells(int32_t num_loops, int32_t num_layers
 LOOPKV_API int32_t loopkv_decode_splits(const loopkv_config* cfg, int32_t kind, int32_t batch,
                              int32_t max_seq_len);
 
+/*
+ * Self-test of the device's bounded waits: one kernel waits on an mbarrier
+ * whose phase never completes.  The wait gives up after the kernels' fixed
+ * limit (2 s by the global timer), ORs LOOPKV_DEVERR_TIMEOUT into *err_flag
+ * and the kernel exits; the context stays usable.  *elapsed_ns receives the
+ * time the wait took.  Both pointers are device memory; the call returns at
+ * once (the kernel runs on the stream).  Errors: INVALID_ARG for null
+ * pointers, CUDA for a failed launch.
+ */
+LOOPKV_API loopkv_status loopkv_selftest_wait_timeout(int32_t* err_flag, uint64_t* elapsed_ns, void* stream);
+
 /* Static text for a status code. */
 LOOPKV_API const char* loopkv_status_string(loopkv_status status);
 

@@ -31,6 +31,7 @@ from .loopkv import (  # noqa: F401
     loopkv_plan_cells,
     loopkv_quantize_append,
     loopkv_record_bytes,
+    loopkv_selftest_wait_timeout,
     loopkv_status_string,
     mask_words,
 )

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libloopkv.so")
-SOURCES = ["loopkv_api.cu", "append.cu", "decode.cu", "planner.cpp"]
+SOURCES = ["loopkv_api.cu", "append.cu", "decode.cu", "planner.cpp", "selftest.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -66,6 +66,7 @@ def _load():
         "loopkv_decode_splits": (I32, [P(loopkv_config), I32, I32, I32]),
         "loopkv_plan_cells": (ctypes.c_int, [I32, I32, VP, I32, I32, I32, VP, VP]),
         "loopkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "loopkv_selftest_wait_timeout": (ctypes.c_int, [VP, VP, VP]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -270,3 +271,13 @@ def loopkv_plan_cells(damage, damage_budget: int, storage_budget: int, q4_read_b
 
 def mask_words(kv: KVCells) -> int:
     return math.ceil(kv.max_blocks_per_seq * kv.block_size / 32)
+
+
+def loopkv_selftest_wait_timeout(err_flag, elapsed_ns, stream=None):
+    """Run the bounded-wait self-test: err_flag int32[1] and elapsed_ns
+    int64[1] on the device receive LOOPKV_DEVERR_TIMEOUT and the wait's
+    duration (about 2 s)."""
+    st = _lib.loopkv_selftest_wait_timeout(_ptr(err_flag, "err_flag", torch.int32),
+                                           _ptr(elapsed_ns, "elapsed_ns", torch.int64), _stream(stream))
+    if st:
+        raise LoopKVError(st, "loopkv_selftest_wait_timeout")

@@ -12,6 +12,18 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+def pytest_sessionstart(session):
+    """Build libloopkv.so (nvcc, sm_100a) when a source is newer than it, so
+    that a fresh checkout tests what it builds.  The build module is loaded
+    from its file: importing the package needs the library first."""
+    import importlib.util
+    path = os.path.join(ROOT, "mixed_precision_kv_loopkv_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_loopkv_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")

@@ -16,9 +16,7 @@ CODE = {"q4": 0, "q2": 1, "reuse": 2}
 
 @pytest.fixture(scope="module")
 def m():
-    from mixed_precision_kv_loopkv_b200 import build as B
-    B.build()
-    import mixed_precision_kv_loopkv_b200 as pkg
+    import mixed_precision_kv_loopkv_b200 as pkg  # built at session start (conftest)
     return pkg
 
 
