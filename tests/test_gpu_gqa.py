@@ -148,3 +148,16 @@ def test_grouped_looped_step():
                  pool_factor=1.3, seed=47, temperature=4.0)
     rep = step_parity(w, nseq=4)
     assert len(rep) == 6
+
+
+def test_grouped_maximum_context():
+    """The largest context the ABI accepts (65536 tokens) with eight query
+    heads per KV head: two splits of 1024 groups, one CTA's shared memory
+    holding 128 KB of logits; sampled heads against the oracle."""
+    lens = [65536, 777]
+    w, kv, data, table, lens_d = _store("q4", 128, lens, 8, 1, seed=48)
+    q = query_for(w, 0, temperature=6.0)
+    out, sm, sc = _decode(kv, q, table, lens_d, 0.01, max_seq_len=65536)
+    check_cell(kv, ["q4"], 0, data, q, table, lens_d, 0.01, 1.0, [(0, 0), (0, 5), (1, 3)],
+               out=out, sel_mask=sm, sel_count=sc)
+    assert int(sc[0, 0]) > 0
