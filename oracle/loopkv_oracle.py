@@ -28,6 +28,10 @@ the readings the library documents:
   * grouped queries (several query heads per KV head): a token's low plane
     is fetched when any head of the group selects it and then serves every
     head of the group;
+  * a reuse cell of a loop before the last may attend, besides the final
+    loop's stored tokens, the current token exactly as its own loop computed
+    it (that token's K/V exist in the loop but are stored nowhere): one more
+    softmax entry with exact key and value and no low plane;
   * attention itself is evaluated in fp64.
 
 Byte layout (the oracle's own reading of the record format, used only to
@@ -37,6 +41,9 @@ compare the library's packed bytes): per (physical block, head) record of
   2-bit: [K plane][K meta][V plane][V meta]
   bf16 : [K rows][V rows]
 A plane row is one token, channel c at byte c // 4, bits 2 * (c % 4) and up.
+The K planes and the V lo plane store the 16 rows one after another
+(row-major); the V hi plane (4-bit) and the V plane (2-bit) store the same
+bytes transposed (column-major): byte 16 * (c // 4) + t is row t's byte c // 4.
 K meta holds (scale, min) bf16 pairs of half the channels of the 32-token
 group: channels [0, D/2) in the group's even block, [D/2, D) in the odd one.
 V meta holds (scale, min) per token row and 32-channel group.
@@ -187,29 +194,45 @@ def select_low_plane(p, tau: float, unit: int = 1) -> np.ndarray:
     return np.repeat(any_in_unit, unit)[:n]
 
 
-def attend(q, k_hat, v_full, v_high, tau: float, sm_scale: float, unit: int = 1):
+def attend(q, k_hat, v_full, v_high, tau: float, sm_scale: float, unit: int = 1, k_cur=None, v_cur=None):
     """Decode attention of one query (``unit``: selection granularity, see
     select_low_plane).
 
     ``v_high`` is None for cells without a low plane (2-bit, bf16); then every
-    token uses ``v_full`` and nothing is selected.  Returns (o fp64[D],
-    selected bool[n], p fp64[n]).
+    token uses ``v_full`` and nothing is selected.
+
+    ``k_cur``, ``v_cur`` (optional, exact rows [D]) add one token after the n
+    stored ones: the current token as its own loop computed it, which a reuse
+    cell has not stored anywhere (it reads the final loop's cell, where that
+    token does not exist yet).  It takes part in the softmax with its exact
+    key and value and has no low plane; the selection rule applies to the
+    stored tokens with their weights in that softmax.
+
+    Returns (o fp64[D], selected bool[n], p fp64[n], or [n + 1] with the
+    current token's weight last).
     """
     k_hat = np.asarray(k_hat, np.float64)
     n, d = k_hat.shape
-    if n == 0:
+    cur = k_cur is not None
+    if n == 0 and not cur:
         return np.zeros(d), np.zeros(0, dtype=bool), np.zeros(0)
-    _, p = softmax_weights(q, k_hat, sm_scale)
+    keys = np.vstack([k_hat, np.asarray(k_cur, np.float64)[None]]) if cur else k_hat
+    _, p = softmax_weights(q, keys, sm_scale)
+    ps = p[:n]
     if v_high is None:
         sel = np.zeros(n, dtype=bool)
-        v_hat = np.asarray(v_full, np.float64)
+        v_hat = np.asarray(v_full, np.float64).reshape(n, d)
     else:
-        sel = select_low_plane(p, tau, unit)
-        v_hat = np.where(sel[:, None], v_full, v_high)
-    return p @ v_hat, sel, p
+        sel = select_low_plane(ps, tau, unit)
+        v_hat = np.where(sel[:, None], v_full, v_high).reshape(n, d)
+    o = ps @ v_hat
+    if cur:
+        o = o + p[n] * np.asarray(v_cur, np.float64)
+    return o, sel, p
 
 
-def attend_grouped(queries, k_hat, v_full, v_high, tau: float, sm_scale: float, unit: int = 1):
+def attend_grouped(queries, k_hat, v_full, v_high, tau: float, sm_scale: float, unit: int = 1,
+                   k_cur=None, v_cur=None):
     """Decode attention of the G query heads that share one KV head.
 
     Grouped-query form of the low-plane rule (the survey's selection
@@ -218,24 +241,31 @@ def attend_grouped(queries, k_hat, v_full, v_high, tau: float, sm_scale: float, 
     fp32 weight, or its unit's largest one, reaches tau), and a fetched row
     serves every head of the group.  So each head's values are the full 4-bit
     values on the union of the heads' selections and the high-plane midpoints
-    elsewhere, while each head keeps its own softmax weights.  Returns
-    (o fp64[G, D], selected bool[n], p fp64[G, n]).
+    elsewhere, while each head keeps its own softmax weights.  ``k_cur``,
+    ``v_cur``: one exact current token of the KV head, as in attend.  Returns
+    (o fp64[G, D], selected bool[n], p fp64[G, n] or [G, n + 1]).
     """
     queries = np.asarray(queries, np.float32)
     g = queries.shape[0]
     k_hat = np.asarray(k_hat, np.float64)
     n, d = k_hat.shape
-    if n == 0:
+    cur = k_cur is not None
+    if n == 0 and not cur:
         return np.zeros((g, d)), np.zeros(0, dtype=bool), np.zeros((g, 0))
-    p = np.stack([softmax_weights(qh, k_hat, sm_scale)[1] for qh in queries])
+    keys = np.vstack([k_hat, np.asarray(k_cur, np.float64)[None]]) if cur else k_hat
+    p = np.stack([softmax_weights(qh, keys, sm_scale)[1] for qh in queries])
+    ps = p[:, :n]
     sel = np.zeros(n, dtype=bool)
     if v_high is None:
-        v_hat = np.asarray(v_full, np.float64)
+        v_hat = np.asarray(v_full, np.float64).reshape(n, d)
     else:
         for h in range(g):
-            sel |= select_low_plane(p[h], tau, unit)
-        v_hat = np.where(sel[:, None], v_full, v_high)
-    return p @ v_hat, sel, p
+            sel |= select_low_plane(ps[h], tau, unit)
+        v_hat = np.where(sel[:, None], v_full, v_high).reshape(n, d)
+    o = ps @ v_hat
+    if cur:
+        o = o + p[:, n:] * np.asarray(v_cur, np.float64)[None]
+    return o, sel, p
 
 
 class StoredSequence:
@@ -254,22 +284,25 @@ class StoredSequence:
         else:
             raise ValueError(kind)
 
-    def attend(self, q, tau: float, sm_scale: float, unit: int = 1):
-        """Attention of one query over every stored token."""
+    def attend(self, q, tau: float, sm_scale: float, unit: int = 1, k_cur=None, v_cur=None):
+        """Attention of one query over every stored token (and the exact
+        current token k_cur, v_cur when given; see attend)."""
         if self.kind == "bf16":
-            return attend(q, self.k_exact, self.v_exact, None, tau, sm_scale)
+            return attend(q, self.k_exact, self.v_exact, None, tau, sm_scale, k_cur=k_cur, v_cur=v_cur)
         k_hat = self.qk.dequant()
         v_full = self.qv.dequant_full()
         v_high = self.qv.dequant_high() if self.kind == "q4" else None
-        return attend(q, k_hat, v_full, v_high, tau, sm_scale, unit)
+        return attend(q, k_hat, v_full, v_high, tau, sm_scale, unit, k_cur=k_cur, v_cur=v_cur)
 
-    def attend_grouped(self, queries, tau: float, sm_scale: float, unit: int = 1):
+    def attend_grouped(self, queries, tau: float, sm_scale: float, unit: int = 1, k_cur=None, v_cur=None):
         """Attention of the G query heads sharing this KV head (see
         attend_grouped)."""
         if self.kind == "bf16":
-            return attend_grouped(queries, self.k_exact, self.v_exact, None, tau, sm_scale)
+            return attend_grouped(queries, self.k_exact, self.v_exact, None, tau, sm_scale, k_cur=k_cur,
+                                  v_cur=v_cur)
         v_high = self.qv.dequant_high() if self.kind == "q4" else None
-        return attend_grouped(queries, self.qk.dequant(), self.qv.dequant_full(), v_high, tau, sm_scale, unit)
+        return attend_grouped(queries, self.qk.dequant(), self.qv.dequant_full(), v_high, tau, sm_scale, unit,
+                              k_cur=k_cur, v_cur=v_cur)
 
 
 def resolve_source(plan, cell: int, num_layers: int) -> int:
@@ -284,11 +317,14 @@ def resolve_source(plan, cell: int, num_layers: int) -> int:
 
 
 def decode_cell(plan, num_layers: int, cell: int, stored: dict, q, seq_lens,
-                tau: float, sm_scale: float, pairs=None):
+                tau: float, sm_scale: float, pairs=None, current=None):
     """Decode attention of one cell for the (b, h) pairs given.
 
     ``stored[(src_cell, b, h)]`` is the StoredSequence of a stored cell;
-    ``q`` is fp32[B, H, D]; returns {(b, h): (o, selected, p)}.
+    ``q`` is fp32[B, H, D]; ``current`` (optional) maps (b, h) to the exact
+    (k, v) rows of the current token, attended after the stored tokens (a
+    reuse cell's own K/V of the token being decoded); returns
+    {(b, h): (o, selected, p)}.
     """
     src = resolve_source(plan, cell, num_layers)
     out = {}
@@ -296,7 +332,8 @@ def decode_cell(plan, num_layers: int, cell: int, stored: dict, q, seq_lens,
         seq = stored[(src, b, h)]
         if int(seq_lens[b]) != seq.n:
             raise ValueError("sequence length does not match the stored sequence")
-        out[(b, h)] = seq.attend(np.asarray(q[b, h], np.float32), tau, sm_scale)
+        kc, vc = (None, None) if current is None else current[(b, h)]
+        out[(b, h)] = seq.attend(np.asarray(q[b, h], np.float32), tau, sm_scale, k_cur=kc, v_cur=vc)
     return out
 
 
@@ -340,6 +377,16 @@ def pack_plane(codes2) -> np.ndarray:
     return (c4[..., 0] | (c4[..., 1] << 2) | (c4[..., 2] << 4) | (c4[..., 3] << 6)).astype(np.uint8)
 
 
+def pack_plane_columns(codes2, block: int = BLOCK) -> np.ndarray:
+    """2-bit codes uint8[block, D] of one block -> column-major plane bytes
+    uint8[D/4 * block]: the row-major plane transposed, so that byte
+    block * j + t is row t's byte j (channels 4j .. 4j + 3)."""
+    rows = pack_plane(codes2)                       # [block, D/4]
+    if rows.shape[0] != block:
+        raise ValueError("a column-major plane holds exactly one block of rows")
+    return np.ascontiguousarray(rows.T).reshape(-1)
+
+
 def _meta_bytes(scale, minv) -> np.ndarray:
     """(scale, min) bf16 pairs, little-endian, scale first -> uint8[..., 4]."""
     s = bf16_bits(scale).astype(np.uint32)
@@ -377,18 +424,21 @@ def sequence_records(kind: str, k, v, block: int = BLOCK):
 
     bits = BITS[kind]
     qk, qv = QuantKeys(k, bits), QuantValues(v, bits)
-    # values: every token
+    # values: every token; the high (2-bit: only) plane column-major
     vmeta = _meta_bytes(qv.scale, qv.minv)          # [n, d/32, 4]
-    if kind == "q4":
-        v_hi, v_lo = pack_plane(qv.codes >> 2), pack_plane(qv.codes & 3)
-    else:
-        v_hi, v_lo = pack_plane(qv.codes), None
+    hi_codes = (qv.codes >> 2) if kind == "q4" else qv.codes
+    v_lo = pack_plane(qv.codes & 3) if kind == "q4" else None
     for t in range(n):
         blk, r = t // block, t % block
-        put(blk, "v_hi" if kind == "q4" else "v", r, v_hi[t])
         if v_lo is not None:
             put(blk, "v_lo", r, v_lo[t])
         put(blk, "v_meta", r, vmeta[t])
+    off, size = secs["v_hi" if kind == "q4" else "v"]
+    for blk in range(nblocks):
+        rows = np.zeros((block, d), dtype=np.uint8)          # tokens past n: zero bytes
+        part = hi_codes[blk * block: (blk + 1) * block]
+        rows[: part.shape[0]] = part
+        rec[blk, off: off + size] = pack_plane_columns(rows, block)
     # keys: complete groups only
     ng = n // GROUP
     if kind == "q4":

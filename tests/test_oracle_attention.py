@@ -369,3 +369,128 @@ def test_grouped_special_cases_and_bounds():
     # an empty sequence gives zeros for every head
     e = O.attend_grouped(qs, np.zeros((0, 128)), np.zeros((0, 128)), np.zeros((0, 128)), 0.01, 1.0)
     assert e[0].shape == (4, 128) and not e[0].any() and e[1].size == 0
+
+
+# ---- the current token of a reuse cell's own loop: one exact extra entry of
+#      the softmax after the stored tokens (no low plane).  Pinned by torch's
+#      attention over the concatenated cache, the decomposition with torch's
+#      softmax over n + 1 tokens, scalar loops and the one-token case.
+
+def _current(seed, d=128, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return _bf16(rng, (d,), scale), _bf16(rng, (d,))
+
+
+@pytest.mark.parametrize("kind", ["q4", "q2", "bf16"])
+@pytest.mark.parametrize("tau", [0.0, math.inf])
+def test_current_token_limits_are_attention_over_concatenation(kind, tau):
+    q, k, v, seq = _case(31, n=211, kind=kind, q_scale=2.0)
+    kc, vc = _current(32, scale=3.0)
+    o, sel, p = seq.attend(q, tau, 1.0, k_cur=kc, v_cur=vc)
+    assert sel.size == 211 and p.size == 212
+    if kind == "bf16":
+        kh, vx = k, v
+    else:
+        kh = seq.qk.dequant()
+        vx = seq.qv.dequant_full() if (kind == "q2" or tau == 0.0) else seq.qv.dequant_high()
+    ref = _sdpa(q, np.vstack([kh, kc[None]]), np.vstack([vx, vc[None]]), 1.0)
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-12)
+    if kind == "q4":
+        assert sel.all() == (tau == 0.0) and (not sel.any()) == (tau == math.inf)
+
+
+@pytest.mark.parametrize("tau", [1e-3, 1e-2, 5e-2])
+def test_current_token_general_tau_decomposition(tau):
+    q, k, v, seq = _case(33, n=400, q_scale=3.0)
+    kc, vc = _current(34, scale=2.0)
+    o, sel, p = seq.attend(q, tau, 1.0, k_cur=kc, v_cur=vc)
+    kh, vf, vh = seq.qk.dequant(), seq.qv.dequant_full(), seq.qv.dequant_high()
+    keys = np.vstack([kh, kc[None]])
+    pt = _torch_p(q, keys, 1.0)
+    np.testing.assert_allclose(p, pt, rtol=1e-12, atol=1e-15)
+    want = pt[:400].astype(np.float32) >= np.float32(tau)
+    np.testing.assert_array_equal(sel, want)
+    ref = _sdpa(q, keys, np.vstack([vh, vc[None]]), 1.0) + (pt[:400][want, None] * (vf - vh)[want]).sum(axis=0)
+    np.testing.assert_allclose(o, ref, rtol=1e-10, atol=1e-12)
+    # the extra entry takes weight: the stored tokens' weights sum to 1 - p_cur
+    assert 0 < p[400] < 1 and abs(p[:400].sum() + p[400] - 1) < 1e-12
+
+
+def test_current_token_alone_is_its_value():
+    o, sel, p = O.attend(np.ones(64), np.zeros((0, 64)), np.zeros((0, 64)), np.zeros((0, 64)), 0.01, 1.0,
+                         k_cur=np.full(64, 0.5), v_cur=np.arange(64.0))
+    assert sel.size == 0 and p.tolist() == [1.0]
+    np.testing.assert_array_equal(o, np.arange(64.0))
+
+
+def test_current_token_brute_force_tiny_loops():
+    """Scalar loops (math.exp, Python floats) over the stored tokens and the
+    current one on a tiny 4-bit case."""
+    rng = np.random.default_rng(35)
+    n, d, tau = 37, 32, 0.03
+    k, v = _bf16(rng, (n, d)), _bf16(rng, (n, d))
+    q = _bf16(rng, (d,), 2.0)
+    kc, vc = _bf16(rng, (d,), 2.0), _bf16(rng, (d,))
+    seq = O.StoredSequence("q4", k, v)
+    o, sel, _ = seq.attend(q, tau, 1.0, k_cur=kc, v_cur=vc)
+    qk, qv = seq.qk, seq.qv
+    logits = []
+    for t in range(n):
+        acc = 0.0
+        for c in range(d):
+            kv = float(qk.minv[0, c]) + float(qk.scale[0, c]) * int(qk.codes[t, c]) if t < 32 else float(k[t, c])
+            acc += float(q[c]) * kv
+        logits.append(acc)
+    logits.append(sum(float(q[c]) * float(kc[c]) for c in range(d)))
+    m = max(logits)
+    e = [math.exp(s - m) for s in logits]
+    z = sum(e)
+    out = [0.0] * d
+    for t in range(n):
+        p = e[t] / z
+        take_low = np.float32(p) >= np.float32(tau)
+        assert take_low == sel[t]
+        for c in range(d):
+            code = int(qv.codes[t, c])
+            s, mn = float(qv.scale[t, 0]), float(qv.minv[t, 0])
+            out[c] += p * (mn + s * (code if take_low else 4 * (code >> 2) + 1.5))
+    for c in range(d):
+        out[c] += e[n] / z * float(vc[c])
+    np.testing.assert_allclose(o, out, rtol=1e-11, atol=1e-13)
+
+
+@pytest.mark.parametrize("g", [2, 4])
+def test_current_token_grouped_union(g):
+    q, k, v, seq = _case(36, n=300)
+    qs = _queries(37, g)
+    kc, vc = _current(38, scale=3.0)
+    tau = 0.01
+    o, sel, p = seq.attend_grouped(qs, tau, 1.0, k_cur=kc, v_cur=vc)
+    kh, vf, vh = seq.qk.dequant(), seq.qv.dequant_full(), seq.qv.dequant_high()
+    keys = np.vstack([kh, kc[None]])
+    pt = [_torch_p(qs[h], keys, 1.0) for h in range(g)]
+    want = np.array([any(np.float32(pt[h][t]) >= np.float32(tau) for h in range(g)) for t in range(300)])
+    np.testing.assert_array_equal(sel, want)
+    for h in range(g):
+        ref = _sdpa(qs[h], keys, np.vstack([vh, vc[None]]), 1.0) + (pt[h][:300][sel, None] * (vf - vh)[sel]).sum(0)
+        np.testing.assert_allclose(o[h], ref, rtol=1e-10, atol=1e-12)
+    # one head: the grouped form is the single-query form
+    o1, s1, p1 = seq.attend(qs[0], tau, 1.0, k_cur=kc, v_cur=vc)
+    og, sg, pg = seq.attend_grouped(qs[:1], tau, 1.0, k_cur=kc, v_cur=vc)
+    np.testing.assert_array_equal(o1, og[0])
+    np.testing.assert_array_equal(s1, sg)
+
+
+def test_reuse_cell_attends_the_current_token():
+    rng = np.random.default_rng(39)
+    N, n, d = 2, 70, 64
+    plan = ["reuse", "q2", "q4", "q4"]
+    stored = {(c, 0, 0): O.StoredSequence(plan[c], _bf16(rng, (n, d)), _bf16(rng, (n, d))) for c in (1, 2, 3)}
+    q = _bf16(rng, (1, 1, d), 2.0)
+    kc, vc = _bf16(rng, (d,), 2.0), _bf16(rng, (d,))
+    got = O.decode_cell(plan, N, 0, stored, q, [n], 0.02, 1.0, pairs=[(0, 0)], current={(0, 0): (kc, vc)})
+    want = stored[(2, 0, 0)].attend(q[0, 0], 0.02, 1.0, k_cur=kc, v_cur=vc)
+    for a, b in zip(got[(0, 0)], want):
+        np.testing.assert_array_equal(a, b)
+    plain = stored[(2, 0, 0)].attend(q[0, 0], 0.02, 1.0)
+    assert not np.allclose(got[(0, 0)][0], plain[0])

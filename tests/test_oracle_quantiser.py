@@ -191,6 +191,16 @@ def test_sequence_records_read_back(kind):
         off, sz = secs[name]
         return O.unpack_plane(rec[blk, off: off + sz].reshape(16, d // 4), d)
 
+    def column_plane(blk, name):
+        # column-major: byte 16 * j + r holds row r's channels 4j .. 4j + 3
+        off, sz = secs[name]
+        b = rec[blk, off: off + sz]
+        out = np.zeros((16, d), dtype=np.uint8)
+        for r in range(16):
+            for c in range(d):
+                out[r, c] = (int(b[16 * (c // 4) + r]) >> (2 * (c % 4))) & 3
+        return out
+
     def meta(blk, name):
         off, sz = secs[name]
         w = rec[blk, off: off + sz].copy().view("<u4")
@@ -201,9 +211,9 @@ def test_sequence_records_read_back(kind):
     for t in range(n):
         blk, r = divmod(t, 16)
         if kind == "q4":
-            vc = plane(blk, "v_hi")[r] * 4 + plane(blk, "v_lo")[r]
+            vc = column_plane(blk, "v_hi")[r] * 4 + plane(blk, "v_lo")[r]
         else:
-            vc = plane(blk, "v")[r]
+            vc = column_plane(blk, "v")[r]
         np.testing.assert_array_equal(vc, qv.codes[t])
         s, m = meta(blk, "v_meta")
         np.testing.assert_array_equal(s.reshape(16, d // 32)[r], qv.scale[t])
@@ -232,3 +242,19 @@ def test_bf16_records_are_raw_rows():
     assert resid is None and rec.shape == (2, O.record_bytes("bf16", 64))
     kr = rec[1, : 16 * 128].copy().view("<u2").reshape(16, 64)
     np.testing.assert_array_equal(kr[3], torch.from_numpy(k[19]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+
+
+def test_column_major_plane_worked_example():
+    """A hand-worked column-major plane: channel c of row t is code
+    (t + c) % 4; byte 16 j + t packs channels 4j .. 4j + 3 of row t LSB first,
+    i.e. codes (t + 4j) % 4, (t + 4j + 1) % 4, ... = t % 4, (t+1) % 4, ..."""
+    d = 8
+    codes = np.array([[(t + c) % 4 for c in range(d)] for t in range(16)], dtype=np.uint8)
+    b = O.pack_plane_columns(codes)
+    assert b.shape == (d // 4 * 16,)
+    for j in range(d // 4):
+        for t in range(16):
+            a = [(t + 4 * j + f) % 4 for f in range(4)]
+            assert b[16 * j + t] == a[0] | a[1] << 2 | a[2] << 4 | a[3] << 6
+    # row 1 of column 0: codes 1, 2, 3, 0 -> 0b00111001
+    assert b[1] == 0x39
