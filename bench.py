@@ -49,7 +49,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mine", choices=["mine", "reference"])
-    ap.add_argument("--workload", default="ouro_step")
+    ap.add_argument("--workload", default="throughput")
     ap.add_argument("--splits", type=int, default=0, help="decode splits override (0 = automatic)")
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--select-unit", type=int, default=1, choices=[1, 16, 32],
@@ -262,18 +262,20 @@ def setup(w, pdl: bool, splits: int, extra: int = 64, ncells: int = 0, fused: bo
     if int(err):
         raise RuntimeError(f"prefill flagged device error {int(err)}")
     q_all = torch.stack([cell_query(w, *divmod(c, w.num_layers), device="cuda") for c in range(C)])
-    kn_all = torch.empty((len(stored), w.batch, 1, w.kv_heads, w.head_dim), dtype=torch.bfloat16,
+    # the current token's K/V of every cell's loop: stored cells append it,
+    # reuse cells attend it exactly after the final loop's tokens
+    kn_all = torch.empty((len(run), w.batch, 1, w.kv_heads, w.head_dim), dtype=torch.bfloat16,
                          device="cuda")
     vn_all = torch.empty_like(kn_all)
-    for i, c in enumerate(stored):
+    for i, c in enumerate(run):
         kn_all[i], vn_all[i] = cell_new_token(w, *divmod(c, w.num_layers), device="cuda")
     out_all = torch.zeros_like(q_all)
     sel_all = torch.zeros((C, w.batch, w.num_heads), dtype=torch.int32, device="cuda")
-    slot = {c: i for i, c in enumerate(stored)}
+    slot = {c: i for i, c in enumerate(run)}
     pos = torch.from_numpy(lens).cuda()
     step = LoopedDecodeStep(
         kv, table, pos, [q_all[c] for c in range(C)],
-        {c: kn_all[slot[c]] for c in stored}, {c: vn_all[slot[c]] for c in stored},
+        {c: kn_all[slot[c]] for c in run}, {c: vn_all[slot[c]] for c in run},
         [out_all[c] for c in range(C)], w.tau, w.sm_scale, int(lens.max()) + 1,
         sel_count=[sel_all[c] for c in range(C)], cells=run, fused=fused)
     torch.cuda.synchronize()
@@ -351,10 +353,12 @@ class DecodeOnly:
         s, kv = self.s, self.s.kv
         for cell in s.cells:
             loop, layer = divmod(cell, kv.num_layers)
-            lens = s.pos if kv.plan_codes[cell] == LOOPKV_CELL_REUSE else s.pos_next
+            reuse = kv.plan_codes[cell] == LOOPKV_CELL_REUSE
+            lens = s.pos if reuse else s.pos_next
             loopkv_decode_attention(kv, loop, layer, s.q[cell], s.block_table, lens, s.tau, s.sm_scale,
                                     out=s.out[cell], max_seq_len=s.max_seq_len,
-                                    sel_count=s.sel_count[cell])
+                                    sel_count=s.sel_count[cell], k_cur=s.k_new.get(cell) if reuse else None,
+                                    v_cur=s.v_new.get(cell) if reuse else None)
 
 
 def capture(fn):
@@ -416,35 +420,96 @@ def oracle_decode(seq, q, w):
     return seq.attend_grouped(q, w.tau, w.sm_scale)[1]
 
 
-def run_oracle(items, w, budget_s: float = None, steps: int = None, warmup: int = 0):
-    """Time the oracle's decode over the sample (one item per step, round
-    robin); returns (GB/s, seconds, items run, threads)."""
+def byte_accounting():
+    """The package's byte-accounting module, loaded from its file: the CPU
+    legs must not import the package, whose import maps the CUDA library."""
+    import importlib.util
+    name = "_loopkv_accounting"
+    if name in sys.modules:
+        return sys.modules[name]
+    path = os.path.join(ROOT, "mixed_precision_kv_loopkv_b200", "accounting.py")
+    spec = importlib.util.spec_from_file_location(name, path)
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[name] = mod
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+_POOL_ITEMS, _POOL_W = None, None
+
+
+def _oracle_worker_init(items, w):
+    global _POOL_ITEMS, _POOL_W
+    _POOL_ITEMS, _POOL_W = items, w
     from threadpoolctl import threadpool_limits
-    from mixed_precision_kv_loopkv_b200.accounting import decode_bytes
-    total_bytes, n_run = 0, 0
-    with threadpool_limits(limits=1):
-        torch_threads = torch.get_num_threads()
-        torch.set_num_threads(1)
-        try:
-            for i in range(warmup):
-                kind, seq, q, n = items[i % len(items)]
-                oracle_decode(seq, q, w)
-            t0 = time.perf_counter()
-            i = 0
-            while True:
-                kind, seq, q, n = items[i % len(items)]
-                sel = oracle_decode(seq, q, w)
-                total_bytes += decode_bytes(kind, w.head_dim, n, int(sel.sum())) + (len(q) - 1) * 4 * w.head_dim
-                i += 1
-                el = time.perf_counter() - t0
-                if steps is not None and i >= steps:
-                    break
-                if budget_s is not None and el >= budget_s:
-                    break
-            n_run = i
-        finally:
-            torch.set_num_threads(torch_threads)
-    return total_bytes / el / 1e9, el, n_run, 1
+    threadpool_limits(limits=1)       # one BLAS thread per worker process
+
+
+def _oracle_item_bytes(kind, n, sel, g, d):
+    return byte_accounting().decode_bytes(kind, d, n, int(sel.sum())) + (g - 1) * 4 * d
+
+
+def _oracle_worker_budget(args):
+    """Round robin over the sample from a worker-specific start for
+    budget_s seconds; returns (bytes, decodes, seconds)."""
+    start, budget_s = args
+    items, w = _POOL_ITEMS, _POOL_W
+    total, i = 0, start
+    t0 = time.perf_counter()
+    while True:
+        kind, seq, q, n = items[i % len(items)]
+        sel = oracle_decode(seq, q, w)
+        total += _oracle_item_bytes(kind, n, sel, len(q), w.head_dim)
+        i += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            return total, i - start, el
+
+
+def _oracle_worker_one(index):
+    items, w = _POOL_ITEMS, _POOL_W
+    kind, seq, q, n = items[index % len(items)]
+    sel = oracle_decode(seq, q, w)
+    return _oracle_item_bytes(kind, n, sel, len(q), w.head_dim)
+
+
+def oracle_pool(items, w, workers: int):
+    """A pool of oracle worker processes (spawned, so that it is safe after
+    the GPU arm has initialised CUDA), one per host core."""
+    import multiprocessing as mp
+    return mp.get_context("spawn").Pool(workers, initializer=_oracle_worker_init, initargs=(items, w))
+
+
+def run_oracle_budget(items, w, budget_s: float, workers: int):
+    """Every worker decodes sampled items for budget_s seconds, all at once;
+    returns (GB/s over all workers, seconds, decodes run)."""
+    with oracle_pool(items, w, workers) as pool:
+        pool.map(_oracle_worker_one, range(workers))          # warm-up: imports, first decode
+        res = pool.map(_oracle_worker_budget, [(k, budget_s) for k in range(workers)])
+    total = sum(r[0] for r in res)
+    secs = max(r[2] for r in res)
+    return total / secs / 1e9, secs, sum(r[1] for r in res)
+
+
+def run_oracle_steps(items, w, steps: int, warmup: int, workers: int):
+    """Steps of one decode per worker, all workers at once; each step is
+    timed by the host clock.  Returns (GB/s, seconds, decodes run)."""
+    with oracle_pool(items, w, workers) as pool:
+        for s in range(max(warmup, 1)):
+            pool.map(_oracle_worker_one, range(s * workers, (s + 1) * workers))
+        total = 0
+        t0 = time.perf_counter()
+        for s in range(steps):
+            total += sum(pool.map(_oracle_worker_one, range(s * workers, (s + 1) * workers)))
+        secs = time.perf_counter() - t0
+    return total / secs / 1e9, secs, steps * workers
 
 
 # ----------------------------------------------------------------- arms
@@ -468,23 +533,25 @@ def workload_config(w, world):
 
 
 def reference_arm(args, world, rank):
-    """The oracle as it stands on the host cores, one sampled (cell,
-    sequence, head) decode per step."""
+    """The oracle as it stands on the host cores: every step, one sampled
+    (cell, sequence, head) decode per host core, all cores at once."""
     from workload import get_workload, make_plan, seq_lens_for
     if rank != 0:
         return
     w = apply_overrides(get_workload(args.workload), args)
     plan, lens = make_plan(w), seq_lens_for(w)
     items = oracle_sample(w, plan, lens, n_pairs=16)
-    gbs, secs, n_run, cores = run_oracle(items, w, steps=args.steps, warmup=args.warmup)
+    cores = host_cores()
+    gbs, secs, n_run = run_oracle_steps(items, w, steps=args.steps, warmup=args.warmup, workers=cores)
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(n_run, 1) * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / max(args.steps, 1) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w, 1),
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": f"one (cell, sequence, head) decode per step, round robin over 16 "
-                                   f"seeded pairs of the {w.name} workload"},
+                         "sample": f"one (cell, sequence, head) decode per host core per step ({cores} worker "
+                                   f"processes, one BLAS thread each), round robin over 16 seeded pairs of "
+                                   f"the {w.name} workload"},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -515,7 +582,7 @@ def main_arm(args, world, rank, local):
     sel = S["sel_all"].cpu().numpy()
     bytes_step = step_bytes(plan, w.num_layers, w.num_loops, w.head_dim, w.num_heads, lens + 1, lens, sel,
                             group=w.num_heads // w.kv_heads,
-                            cells=step.cells)
+                            cells=step.cells, reuse_current=True)
     value = aggregate_value(bytes_step * args.steps, world, ms_max / 1e3)
     us_step = ms_max / args.steps * 1e3
 
@@ -549,11 +616,13 @@ def main_arm(args, world, rank, local):
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         items = oracle_sample(w, plan, lens, n_pairs=12)
-        gbs, secs, n_run, cores = run_oracle(items, w, budget_s=args.cpu_seconds, warmup=2)
+        cores = host_cores()
+        gbs, secs, n_run = run_oracle_budget(items, w, budget_s=args.cpu_seconds, workers=cores)
         unit = "head" if w.kv_heads == w.num_heads else f"KV head with its {w.num_heads // w.kv_heads} query heads"
         cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-               "sample": f"{n_run} (cell, sequence, {unit}) decodes over {secs:.1f} s, round robin over "
-                         f"12 seeded pairs of the {w.name} workload (numpy fp64, one BLAS thread)"}
+               "sample": f"{n_run} (cell, sequence, {unit}) decodes over {secs:.1f} s on {cores} worker "
+                         f"processes (one per host core, numpy fp64, one BLAS thread each), round robin over "
+                         f"12 seeded pairs of the {w.name} workload"}
 
     if rank == 0:
         cfg = workload_config(w, world)

@@ -2,6 +2,7 @@
 whole-job aggregate over world_size 2 gloo ranks, plus the reference arm's
 bookkeeping."""
 
+import json
 import os
 import socket
 
@@ -84,3 +85,33 @@ def test_sweep_overrides_and_strict_json():
     assert '"tau": "inf"' in text and "all bf16" in cfg["workload"] and "temperature 4.0" in cfg["workload"]
     plain = bench.apply_overrides(get_workload("ouro_step"), bench.parse_args([]))
     assert plain == get_workload("ouro_step")
+
+
+def test_reference_arm_maps_no_product_library(tmp_path):
+    """The oracle arm (all host cores) runs without importing the package,
+    so the CUDA library never enters its process."""
+    import subprocess
+    import sys
+    code = (
+        "import sys, json; sys.argv = ['bench.py', '--impl', 'reference', '--workload', 'tiny', '--steps', '2', "
+        "'--warmup', '1']\n"
+        "import bench; bench.main()\n"
+        "maps = open('/proc/self/maps').read()\n"
+        "print('LOADED' if 'libloopkv' in maps or 'mixed_precision_kv_loopkv_b200' in sys.modules else 'CLEAN')\n")
+    res = subprocess.run([sys.executable, "-c", code], cwd=bench.ROOT, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = res.stdout.strip().splitlines()
+    assert lines[-1] == "CLEAN", res.stdout
+    line = json.loads(lines[-2])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["cores"] == bench.host_cores()
+
+
+def test_oracle_budget_on_all_cores():
+    """The CPU baseline's worker pool decodes on every host core and counts
+    its bytes with the package's own accounting."""
+    from workload import get_workload, make_plan, seq_lens_for
+    w = get_workload("tiny")
+    items = bench.oracle_sample(w, make_plan(w), seq_lens_for(w), n_pairs=2)
+    gbs, secs, n_run = bench.run_oracle_budget(items, w, budget_s=0.5, workers=2)
+    assert gbs > 0 and secs >= 0.5 and n_run >= 2
