@@ -70,6 +70,11 @@ def parse_args(argv=None):
                     help="store every cell as bf16 (the unquantised comparison run of the tau sweep)")
     ap.add_argument("--kv-heads", type=int, default=0,
                     help="KV heads (grouped queries: the workload's query heads share them; 0 = one per head)")
+    ap.add_argument("--ingest-ncu", default=None, metavar="CSV",
+                    help="write profiles/decode_attention_<workload>.json from an ncu --csv launch log, then exit")
+    ap.add_argument("--ncu-scale", type=float, default=1.0,
+                    help="with --ingest-ncu: factor from the captured launches to the workload's full launch")
+    ap.add_argument("--ncu-command", default="", help="with --ingest-ncu: the command that made the capture")
     return ap.parse_args(argv)
 
 
@@ -208,15 +213,13 @@ def decode_source_hash() -> str:
 
 
 def profiled_fields(workload: str) -> dict:
-    """Machine-read fields of the committed ncu summary of the decode kernel
-    (empty unless it was taken on the current kernel source)."""
-    path = os.path.join(ROOT, "profiles", f"decode_attention_{workload}.md")
+    """Machine-written fields of the committed ncu summary of the decode
+    kernel (profiles/decode_attention_<workload>.json, written by
+    --ingest-ncu); empty unless it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"decode_attention_{workload}.json")
     try:
-        fields = {}
-        for line in open(path):
-            if ":" in line and line.strip().startswith("- "):
-                k, v = line.strip()[2:].split(":", 1)
-                fields[k.strip()] = v.strip().strip("`")
+        with open(path) as f:
+            fields = json.load(f)
         return fields if fields.get("source_sha256") == decode_source_hash() else {}
     except Exception:
         return {}
@@ -226,8 +229,79 @@ def profiled_traffic(workload: str):
     """Per-launch DRAM bytes of the decode kernel from the committed ncu summary."""
     try:
         return float(profiled_fields(workload)["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+    except (KeyError, ValueError, TypeError):
         return None
+
+
+KIND_OF_TEMPLATE = {"0": "q4", "1": "q2", "3": "bf16"}
+
+
+def parse_ncu_csv(path: str):
+    """Per-launch metrics of the decode kernel from an ncu --csv log:
+    [(source kind, {metric: value})] in launch order."""
+    import csv
+    import re
+    rows, hdr = [], None
+    with open(path) as f:
+        for r in csv.reader(f):
+            if r and r[0] == "ID":
+                hdr = r
+                continue
+            if hdr and len(r) == len(hdr):
+                rows.append(dict(zip(hdr, r)))
+    launches = {}
+    for d in rows:
+        if "decode_kernel" not in d["Kernel Name"]:
+            continue
+        m = re.search(r"decode_kernel<(\d+),", d["Kernel Name"])
+        kind = KIND_OF_TEMPLATE.get(m.group(1), "?") if m else "?"
+        ent = launches.setdefault(d["ID"], (kind, {}))
+        try:
+            ent[1][d["Metric Name"]] = float(d["Metric Value"].replace(",", ""))
+        except ValueError:
+            pass
+    return [launches[k] for k in sorted(launches, key=int)]
+
+
+def ingest_ncu(csv_path: str, workload: str, scale: float = 1.0, command: str = "") -> dict:
+    """Plan-weighted per-launch DRAM bytes and warp instructions of the
+    decode kernel for a workload, from the launches of an ncu capture
+    (scaled by ``scale`` when the capture ran a smaller batch); written to
+    profiles/decode_attention_<workload>.json with the kernel source hash."""
+    from workload import get_workload, make_plan
+    w = get_workload(workload)
+    plan = make_plan(w)
+    L, N = w.num_loops, w.num_layers
+    src_kind = [plan[c] if plan[c] != "reuse" else plan[(L - 1) * N + c % N] for c in range(len(plan))]
+    per_kind = {}
+    for kind, m in parse_ncu_csv(csv_path):
+        per_kind.setdefault(kind, []).append(m)
+    out = {"source_sha256": decode_source_hash(), "workload": workload, "capture_scale": scale,
+           "command": command, "per_kind": {}}
+    tot_dram = tot_inst = 0.0
+    weight = 0
+    for kind in sorted(set(src_kind)):
+        ms = per_kind.get(kind)
+        if not ms:
+            raise ValueError(f"no captured launch of a {kind} source")
+        dram = [(m.get("dram__bytes_read.sum", 0) + m.get("dram__bytes_write.sum", 0)) * scale for m in ms]
+        inst = [m.get("smsp__inst_executed.sum", 0) * scale for m in ms]
+        dur = [m.get("gpu__time_duration.sum", 0) * scale for m in ms]
+        cnt = src_kind.count(kind)
+        out["per_kind"][kind] = {"launches_captured": len(ms), "launches_per_step": cnt,
+                                 "dram_bytes_per_launch": sum(dram) / len(ms),
+                                 "warp_instructions_per_launch": sum(inst) / len(ms),
+                                 "duration_ns_per_launch": sum(dur) / len(ms)}
+        tot_dram += cnt * sum(dram) / len(ms)
+        tot_inst += cnt * sum(inst) / len(ms)
+        weight += cnt
+    out["dram_bytes_per_launch"] = tot_dram / weight
+    out["warp_instructions_per_launch"] = tot_inst / weight
+    path = os.path.join(ROOT, "profiles", f"decode_attention_{workload}.json")
+    with open(path, "w") as f:
+        json.dump(out, f, indent=1)
+        f.write("\n")
+    return out
 
 
 # ----------------------------------------------------------------- workload setup
@@ -670,6 +744,9 @@ def main_arm(args, world, rank, local):
 
 def main(argv=None):
     args = parse_args(argv)
+    if args.ingest_ncu:
+        print(json.dumps(ingest_ncu(args.ingest_ncu, args.workload, args.ncu_scale, args.ncu_command), indent=1))
+        return
     world, rank, local = dist_env()
     if args.impl == "reference":
         reference_arm(args, world, rank)

@@ -27,8 +27,13 @@
  *   4-bit : [K hi plane][K lo plane][K meta][V hi plane][V meta][V lo plane]
  *   2-bit : [K plane][K meta][V plane][V meta]
  *   bf16  : [K rows bf16][V rows bf16]
- * plane      = 16 rows of D/4 bytes; channel c of a row at byte c/4,
- *              bits 2*(c%4) and 2*(c%4)+1 (least significant first);
+ * row-major plane (K planes, V lo plane) = 16 rows of D/4 bytes, one row per
+ *              token; channel c of a row at byte c/4, bits 2*(c%4) and
+ *              2*(c%4)+1 (least significant first);
+ * column-major plane (V hi plane, 2-bit V plane) = the same bytes
+ *              transposed: D/4 columns of 16 bytes, byte 16*(c/4) + t holds
+ *              token t's channels 4*(c/4) .. 4*(c/4)+3 (same bit order), so
+ *              that one 32-bit word holds one 4-channel column of 4 tokens;
  * K meta     = (scale, min) bf16 pairs (scale in the low half of each 32-bit
  *              word) of the 32-token key group: channels [0, D/2) in the
  *              group's even block, [D/2, D) in its odd block;
@@ -49,12 +54,14 @@
  *     the optional device word *err_flag as LOOPKV_DEVERR_* bits and the
  *     affected (sequence, head) is skipped (decode writes zeros for it);
  *     kernels never trap;
- *   - the library keeps no global state; concurrent calls on different
+ *   - the library's only global state is host-side launch settings: each
+ *     kernel build's shared-memory limit and cluster permission are set once
+ *     per device, and SM counts and occupancy answers are cached, all behind
+ *     locks; concurrent calls from several host threads or on different
  *     streams are safe as long as they do not write the same cells.
  * Inputs must be finite; the fp32 key arithmetic assumes |q * scale * sm_scale|
- * below 2^40; value scales (max - min of a 32-channel group over 3 or 15) must
- * not exceed 255 (|values| up to about 750 for 2-bit and 3800 for 4-bit cells):
- * the append flags larger ones with LOOPKV_DEVERR_RANGE.
+ * below 2^40.  Value weights are carried in fixed point scaled per warp to
+ * the largest value scale seen, so value scales have no limit of their own.
  */
 #ifndef LOOPKV_H
 #define LOOPKV_H
@@ -92,8 +99,8 @@ typedef enum {
 #define LOOPKV_DEVERR_BLOCK_ID 0x1 /* block-table entry outside [0, num_blocks) */
 #define LOOPKV_DEVERR_SEQ_LEN 0x2  /* length beyond the block table or max_seq_len */
 #define LOOPKV_DEVERR_TIMEOUT 0x4  /* a bounded wait on the device gave up */
-#define LOOPKV_DEVERR_RANGE 0x8    /* a value group's scale exceeds 255: the decode
-                                      kernel's f16 value weights would overflow */
+#define LOOPKV_DEVERR_RANGE 0x8    /* reserved (no longer raised: value scales
+                                      have no limit) */
 
 /* loopkv_config.flags */
 #define LOOPKV_FLAG_PDL 0x1 /* programmatic dependent launch: a kernel may start
@@ -181,29 +188,40 @@ LOOPKV_API loopkv_status loopkv_quantize_append(const loopkv_config* cfg, const 
  * them selects it; it then serves all G heads (their values are full 4-bit
  * on the union of the heads' selections).  sel_mask and sel_count report
  * that union for every head of the group.
+ * The current token (optional k_cur, v_cur): a looped model computes the
+ * current token's K and V in every loop, but a reuse cell stores nothing and
+ * the final loop's cell does not hold that token yet, so a reuse cell of an
+ * earlier loop passes its own loop's rows here.  They join the softmax as one
+ * more token after the seq_lens[b] stored ones, with their exact bf16 key and
+ * value and no low plane; the stored tokens' weights, and so the low-plane
+ * selection, are taken in that softmax (LoopKV abstract: a reuse cell reads
+ * the final loop's KV; the current token's own entry is this library's
+ * reading of causal attention in such a cell).
  *
  *   q           : device bf16 [batch][H][D]
+ *   k_cur, v_cur: optional device bf16 [batch][Hkv][D] (both or neither)
  *   block_table : device int32 [batch][max_blocks_per_seq]
  *   seq_lens    : device int32 [batch], each in [0, max_seq_len]
  *   max_seq_len : host upper bound on seq_lens (sizes the split over the
  *                 context); 0 means max_blocks_per_seq * block_size
  *   tau         : >= 0 or +INF;  sm_scale: logit = sm_scale * q . k
- *   out         : device bf16 [batch][H][D]; zeros where seq_len = 0
+ *   out         : device bf16 [batch][H][D]; zeros where seq_len = 0 and no
+ *                 current token is given
  *   sel_mask    : optional device uint32 [batch][H][W], W = ceil(max_blocks_per_seq
  *                 * block_size / 32); bit t%32 of word t/32 = token t took its low
  *                 plane; words past ceil(seq_len/32) are not written
  *   sel_count   : optional device int32 [batch][H], number of selected tokens
  *   err_flag    : optional device int32
- * Errors: INVALID_ARG for tau < 0 or NaN, null required pointers, batch
- * outside [0, max_batch]; BAD_PLAN; UNSUPPORTED for max_seq_len above 65536,
- * for a 4-bit source with G x decode_splits above 16 (the CTAs of one KV
- * head's query heads and splits form one thread-block cluster), or for a
- * context split too long for one CTA's shared memory.
+ * Errors: INVALID_ARG for tau < 0 or NaN, null required pointers, only one of
+ * k_cur / v_cur, batch outside [0, max_batch]; BAD_PLAN; UNSUPPORTED for
+ * max_seq_len above 65536, for a 4-bit source with G x decode_splits above 16
+ * (the CTAs of one KV head's query heads and splits form one thread-block
+ * cluster), or for a context split too long for one CTA's shared memory.
  */
 LOOPKV_API loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const loopkv_cells* cells,
-                                      int32_t loop, int32_t layer, const void* q,
-                                      const int32_t* block_table, const int32_t* seq_lens,
-                                      int32_t batch, int32_t max_seq_len, float tau,
+                                      int32_t loop, int32_t layer, const void* q, const void* k_cur,
+                                      const void* v_cur, const int32_t* block_table,
+                                      const int32_t* seq_lens, int32_t batch, int32_t max_seq_len, float tau,
                                       float sm_scale, void* out, uint32_t* sel_mask,
                                       int32_t* sel_count, int32_t* err_flag, void* stream);
 
@@ -224,7 +242,7 @@ LOOPKV_API loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const
  * Errors: as loopkv_decode_attention, INVALID_ARG for a reuse cell or
  * null k_new / v_new, and UNSUPPORTED with grouped queries (G > 1: append
  * with loopkv_quantize_append, then decode).  Device faults: LOOPKV_DEVERR_SEQ_LEN for start_pos + 1
- * above max_seq_len or the capacity, BLOCK_ID, RANGE as for the append.
+ * above max_seq_len or the capacity, BLOCK_ID as for the append.
  */
 LOOPKV_API loopkv_status loopkv_append_decode_attention(
     const loopkv_config* cfg, const loopkv_cells* cells, int32_t loop, int32_t layer, const void* k_new,

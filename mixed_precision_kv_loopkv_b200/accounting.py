@@ -38,7 +38,7 @@ def decode_bytes(kind: str, d: int, n: int, n_selected: int = 0) -> int:
 
 
 def step_bytes(plan, num_layers: int, num_loops: int, d: int, heads: int, lens_stored, lens_reuse,
-               selected=None, cells=None, group: int = 1) -> int:
+               selected=None, cells=None, group: int = 1, reuse_current: bool = False) -> int:
     """Bytes of one looped decode step: every cell decodes every (sequence,
     head); stored cells over lens_stored[b] tokens, reuse cells over the
     final loop's lens_reuse[b]; selected[cell][b][h] low-plane rows.
@@ -46,7 +46,9 @@ def step_bytes(plan, num_layers: int, num_loops: int, d: int, heads: int, lens_s
     ``group`` query heads share one KV head (``heads`` counts query heads):
     the KV head's cache, and the low-plane rows of the union of the group's
     selections (reported identically for every head of the group), are
-    counted once per group; queries and outputs once per query head."""
+    counted once per group; queries and outputs once per query head.
+    ``reuse_current``: reuse cells also read the current token's exact bf16
+    K and V row (4 * D bytes per sequence and KV head)."""
     total = 0
     for cell, kind in enumerate(plan):
         if cells is not None and cell not in cells:
@@ -58,4 +60,6 @@ def step_bytes(plan, num_layers: int, num_loops: int, d: int, heads: int, lens_s
             for hk in range(heads // group):
                 sel = 0 if selected is None else int(selected[cell][b][hk * group])
                 total += decode_bytes(src_kind, d, int(n), sel) + (group - 1) * 2 * d * 2
+                if reuse_current and kind == "reuse":
+                    total += 4 * d
     return total

@@ -10,7 +10,7 @@
 //
 // One CTA per (head, sequence):
 //   1. each new value token: four warps quantise its 32-channel groups (one
-//      lane per channel) and write both planes and the (scale, min) word;
+//      lane per channel) and write its planes and the (scale, min) word;
 //   2. every key group completed by this call (its 32nd token arrives):
 //      quantised per channel (one lane per token) from the new tokens and the
 //      exact ones waiting in the key residual; planes and meta written;
@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
       const int pos = start + t;
       const float x = __bfloat162float(vb[t * tok_stride + g * kGroup + lane]);
       uint8_t* rec = t == 0 ? rec_first : record_at<KIND, D>(cell, pos);
-      store_value_group<KIND, D>(rec, pos % kBlock, g, x, lane, p.err);
+      store_value_group<KIND, D>(rec, pos % kBlock, g, x, lane);
     }
 
     // 2. key groups completed by this call: groups [start/32, end/32 - 1]

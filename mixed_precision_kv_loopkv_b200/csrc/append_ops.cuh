@@ -14,9 +14,6 @@
 
 namespace loopkv {
 
-// Largest value-group scale the decode kernel's f16 value weights carry.
-constexpr float kMaxValueScale = 255.f;
-
 __device__ __forceinline__ float warp_min(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
@@ -80,10 +77,12 @@ __device__ __forceinline__ uint8_t* record_at(const CellRows& c, int pos) {
 }
 
 // Value group g of one token (whole warp; x = this lane's channel 32g + lane):
-// both planes of the token's row and its (scale, min) word.  rec may be null
-// (the warp still takes part in the shuffles).
+// its (scale, min) word, its high plane (2-bit cells: its only plane) in the
+// block's column-major layout (byte 16 j + row = the token's channels 4j ..
+// 4j + 3), and for 4-bit cells its low plane in the row-major layout.  rec
+// may be null (the warp still takes part in the shuffles).
 template <int KIND, int D>
-__device__ __forceinline__ void store_value_group(uint8_t* rec, int row, int g, float x, int lane, int32_t* err) {
+__device__ __forceinline__ void store_value_group(uint8_t* rec, int row, int g, float x, int lane) {
   using R = Rec<KIND, D>;
   constexpr int BITS = KIND == LOOPKV_CELL_Q4 ? 4 : 2;
   constexpr bool kSplit = KIND == LOOPKV_CELL_Q4;
@@ -91,19 +90,16 @@ __device__ __forceinline__ void store_value_group(uint8_t* rec, int row, int g, 
   float s_b, mn_b;
   group_params<BITS>(warp_min(x), warp_max(x), s_b, mn_b);
   const uint32_t code = group_code<BITS>(x, s_b, mn_b);
-  const uint32_t shift = 2u * (lane & 15);
-  const uint32_t w_hi = half_warp_or((kSplit ? code >> 2 : code) << shift);
-  const uint32_t w_lo = kSplit ? half_warp_or((code & 3u) << shift) : 0u;
+  // the high plane: 4 channels (lanes) per byte
+  uint32_t byte = (kSplit ? code >> 2 : code) << (2 * (lane & 3));
+  byte |= __shfl_xor_sync(0xffffffffu, byte, 1);
+  byte |= __shfl_xor_sync(0xffffffffu, byte, 2);
+  const uint32_t w_lo = kSplit ? half_warp_or((code & 3u) << (2 * (lane & 15))) : 0u;
   if (!rec) return;
-  if ((lane & 15) == 0) {
-    const int word = 2 * g + (lane >> 4);
-    *reinterpret_cast<uint32_t*>(rec + R::kVHi + row * R::kRow + word * 4) = w_hi;
-    if constexpr (kSplit) *reinterpret_cast<uint32_t*>(rec + R::kQ4VLo + row * R::kRow + word * 4) = w_lo;
-  }
-  if (lane == 0) {
-    *reinterpret_cast<uint32_t*>(rec + R::kVMetaOff + (row * kVGroups + g) * 4) = meta_word(s_b, mn_b);
-    if (s_b > kMaxValueScale) flag_error(err, LOOPKV_DEVERR_RANGE);
-  }
+  if ((lane & 3) == 0) rec[R::kVHi + (g * (kGroup / 4) + lane / 4) * kBlock + row] = static_cast<uint8_t>(byte);
+  if (kSplit && (lane & 15) == 0)
+    *reinterpret_cast<uint32_t*>(rec + R::kQ4VLo + row * R::kRow + (2 * g + (lane >> 4)) * 4) = w_lo;
+  if (lane == 0) *reinterpret_cast<uint32_t*>(rec + R::kVMetaOff + (row * kVGroups + g) * 4) = meta_word(s_b, mn_b);
 }
 
 // Key group G (positions 32G .. 32G + 31), quantised per channel: lane =

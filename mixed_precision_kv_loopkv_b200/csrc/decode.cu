@@ -38,6 +38,9 @@
 #include <limits.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include <cuda_fp16.h>
 
@@ -51,6 +54,7 @@ namespace {
 constexpr int kNW = 4;                 // warps per CTA, each streams its own groups
 constexpr int kThreads = 32 * kNW;
 constexpr int kExpOff = 64;            // E: key products live at 2^-64 of their size
+constexpr size_t kMaxDynamicSmem = 227u * 1024u;  // opt-in dynamic shared memory of one CTA
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 
@@ -107,53 +111,37 @@ __device__ __forceinline__ float2 dot16(const float2* c, uint32_t a, uint32_t b,
   return __fadd2_rn(acc0, acc1);
 }
 
-// acc[p] += w * (codes of channels 2p, 2p+1) of one 16-channel word
-template <bool FOUR>
-__device__ __forceinline__ void axpy16(float2* acc, float2 ww, uint32_t a, uint32_t b) {
-  if constexpr (FOUR) {
-    uint32_t e, o;
-    combine_planes(a, b, e, o);
-    const uint32_t e20 = e >> 20, o20 = o >> 20;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) acc[m] = __ffma2_rn(ww, make_float2(nib(e, e20, m), nib(o, o20, m)), acc[m]);
-  } else {
-    const uint32_t a22 = a >> 22;
-#pragma unroll
-    for (int p = 0; p < 8; ++p)
-      acc[p] = __ffma2_rn(ww, make_float2(fld2(a, a22, 2 * p), fld2(a, a22, 2 * p + 1)), acc[p]);
-  }
-}
-
-// Mixed-precision FMA: fp32 accumulator += f16 x f16 (low / high half of a
-// 32-bit register times the f16 in the low half of w).  The product of two
-// f16 values is exact in fp32.
-__device__ __forceinline__ float fma_h_lo(uint32_t f, uint32_t w, float c) {
-  float d;
-  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
-      "fma.rn.f32.f16 %0, a0, b0, %3;\n\t}"
-      : "=f"(d) : "r"(f), "r"(w), "f"(c));
+// Two-way integer dot products (unsigned): d = c + a.lo16 * b.byte0 + a.hi16 * b.byte1
+// (lo) or ... * b.byte2, b.byte3 (hi).  a packs the fixed-point weights of two
+// tokens, b the 2-bit codes (pre-shifted fields) of four tokens of one channel.
+__device__ __forceinline__ uint32_t dp2a_lo(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("dp2a.lo.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
-__device__ __forceinline__ float fma_h_hi(uint32_t f, uint32_t w, float c) {
-  float d;
-  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
-      "fma.rn.f32.f16 %0, a1, b0, %3;\n\t}"
-      : "=f"(d) : "r"(f), "r"(w), "f"(c));
+__device__ __forceinline__ uint32_t dp2a_hi(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("dp2a.hi.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
-// One AND isolates channel i (i < 8) in the low half and channel i + 8 in the
-// high half of a 2-bit plane word, both as f16 subnormals code * 2^(p - 24),
-// p = 2i for i < 5 and 2(i - 5) after a 10-bit shift for the rest.
-__host__ __device__ constexpr int posh(int i) { return 2 * (i < 5 ? i : i - 5); }
-// acc[i] += w * (channel i, channel i + 8) of one 16-channel word; w is f16.
-__device__ __forceinline__ void axpy16_h(float2* acc, uint32_t wh, uint32_t x) {
-  const uint32_t x10 = x >> 10;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t f = i < 5 ? (x & (0x00030003u << (2 * i))) : (x10 & (0x00030003u << (2 * (i - 5))));
-    acc[i].x = fma_h_lo(f, wh, acc[i].x);
-    acc[i].y = fma_h_hi(f, wh, acc[i].y);
-  }
+// acc[f] += the four tokens' codes of channel 4 col + f, weighted by the two
+// weight pairs a01 (tokens 0, 1 of the word) and a23 (tokens 2, 3).  Byte t
+// of w holds token t's channels 4 col .. 4 col + 3 at bits 0-1, 2-3, 4-5,
+// 6-7; fields 2 and 3 are read from w >> 4, so every field is isolated by one
+// AND and carries a factor 1 (f even) or 4 (f odd), undone at the end.
+__device__ __forceinline__ void column_dot(uint32_t* acc, uint32_t w, uint32_t a01, uint32_t a23) {
+  const uint32_t y = w >> 4;
+  const uint32_t x0 = w & 0x03030303u, x1 = w & 0x0C0C0C0Cu;
+  const uint32_t x2 = y & 0x03030303u, x3 = y & 0x0C0C0C0Cu;
+  acc[0] = dp2a_hi(a23, x0, dp2a_lo(a01, x0, acc[0]));
+  acc[1] = dp2a_hi(a23, x1, dp2a_lo(a01, x1, acc[1]));
+  acc[2] = dp2a_hi(a23, x2, dp2a_lo(a01, x2, acc[2]));
+  acc[3] = dp2a_hi(a23, x3, dp2a_lo(a01, x3, acc[3]));
+}
+// Round a non-negative float below 2^22 to the nearest integer in the low
+// bits of the result (added to 1.5 * 2^23, whose unit in the last place is 1).
+__device__ __forceinline__ uint32_t round_fixed(float w, float s) {
+  return __float_as_uint(fmaf(w, s, 12582912.f));
 }
 
 // Index of the sequence with rank r when the batch is ordered by decreasing
@@ -211,7 +199,7 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, int b, int h
           reinterpret_cast<const uint4*>(value ? vb : kb)[c];
     }
   } else {
-    if (warp < D / kGroup) store_value_group<KIND, D>(rec, row, warp, __bfloat162float(vb[warp * kGroup + lane]), lane, p.err);
+    if (warp < D / kGroup) store_value_group<KIND, D>(rec, row, warp, __bfloat162float(vb[warp * kGroup + lane]), lane);
     __nv_bfloat16* res = p.wr_residual + (static_cast<size_t>(b) * p.Hkv + h) * kGroup * D;
     if (pos % kGroup == kGroup - 1) {
       store_key_group<KIND, D>(cell, pos / kGroup, lane == kGroup - 1 ? kb : res + lane * D, warp, lane, kNW);
@@ -233,26 +221,30 @@ struct Cfg {
   static constexpr int kHalf = kLoad + 64;
   static constexpr int kStage = kHalf + kLoad;
   static constexpr int kNSW = 2;                           // ring stages per warp
+  // keys: lane (r, k) takes channels kCW*k .. kCW*k + kCW - 1 of tokens r + 8j
   static constexpr int kCH = 4;                            // lanes per token
   static constexpr int kCW = D / kCH;                      // channels per lane
   static constexpr int kNWRD = kCW / 16;                   // plane words per lane and token
   static constexpr int kTS = 32 / kCH;                     // token sub-groups per warp
   static constexpr int kTPL = 32 / kTS;                    // tokens per lane per group
   static constexpr int kE = kQuant ? kExpOff : 0;
-  // 2-bit value fields go through f16 x f16 -> fp32 FMAs; the full 4-bit
-  // values of the tau = 0 variant and bf16 cells stay on FP32x2 FMAs
-  static constexpr bool kHalfV = kQuant && !FULLV;
-  // power of two folded into the softmax weight for the value products
-  // (half path: weights <= 2^6 keep value scales up to 2^9 inside f16)
-  static constexpr int kVSh = !kQuant ? 0 : kHalfV ? 6 : 85;
+  // values: the plane is column-major within a block; lane (hb, col) takes
+  // the 4 channels of column col (of the block hb for D = 64, of both blocks
+  // for D = 128) for every token
+  static constexpr int kCols = D / 4;                      // 4-channel columns
+  static constexpr int kLPC = 32 / kCols;                  // lanes per column (1 or 2)
+  static constexpr int kVG = D / kGroup;                   // value groups per token
   static constexpr bool kLogits = kQ4 && !FULLV;           // pass 2 needs the logits
   static constexpr bool kFourV = kQ4 && FULLV;             // full 4-bit values in pass 1
+  // the streamed value codes count 4 x hi for a 4-bit cell: fixed-point
+  // weights are scaled for 4 x scale
+  static constexpr float kMult = kQ4 ? 4.f : 1.f;
 };
 
 // Shared-memory carve-up (bytes), identical on host and device.
-// After pass 1 a warp's ring is idle and holds the warp's results: the
-// per-channel partial sums of its TS token sub-groups (wscr, at the ring's
-// start) and its low-plane corrections (after them).  The exchange area (xchg) is never aliased: peers of the
+// After pass 1 a warp's ring is idle and holds the warp's results: its
+// per-channel sums (wres, at the ring's start) and its low-plane corrections
+// (after them).  The exchange area (xchg) is never aliased: peers of the
 // cluster store into it while this CTA may still be in pass 1.
 //   xchg: table float4[8 * kNW] (every warp's max, sum, error bits),
 //         red float[D] (the owner's slice sums of every split),
@@ -260,14 +252,19 @@ struct Cfg {
 struct Smem {
   size_t rings, ring_bytes, bars, qconst, q2buf, logits, ids, masks, xchg, scal, total;
 };
+// Per-warp buffer of 512 B, used twice per group: the key coefficients (128
+// floats) while the keys are read, then the group's value weights
+// (fixed-point u16 [2][D/32][32]: high and, for full 4-bit values, low plane;
+// fp32 [32] for bf16 cells) once every lane has its logit.
+constexpr int kWarpBufBytes = 512;
 __host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int d, bool logits) {
   Smem s;
   s.rings = 0;
   s.ring_bytes = static_cast<size_t>(stage_bytes) * nsw;
   s.bars = s.rings + s.ring_bytes * kNW;
   s.qconst = s.bars + 8 * nsw * kNW;                       // qf[D], qs[D]
-  s.q2buf = s.qconst + static_cast<size_t>(8) * d;         // per warp: 128 floats, swizzled
-  s.logits = s.q2buf + static_cast<size_t>(4) * 128 * kNW;
+  s.q2buf = s.qconst + static_cast<size_t>(8) * d;         // per warp: kWarpBufBytes
+  s.logits = s.q2buf + static_cast<size_t>(kWarpBufBytes) * kNW;
   s.ids = s.logits + (logits ? 128 * static_cast<size_t>(cg) : 0);  // two block ids per group
   s.masks = s.ids + (logits ? 8 * static_cast<size_t>(cg) : 0);     // selection word per group
   s.xchg = s.masks + (logits ? 4 * static_cast<size_t>(cg) : 0);
@@ -280,19 +277,27 @@ __host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int 
 // Per-CTA scalar slots.
 enum { kSlotBad = 0, kSlotCnt0 = 4 };
 
-// 16-byte piece (of CW / 4) where lane (r, k) stores channels 4v .. 4v + 3
-// of its chunk: the rotation by 2k + r puts the eight lanes of each store
-// phase on distinct bank groups (CW = 32).
-template <int CW>
-__host__ __device__ __forceinline__ int wscr_piece(int v, int k, int r) {
-  return (v + 2 * k + r) & (CW / 4 - 1);
-}
+// Largest exponent F of the fixed-point value weights (their scale before
+// the first group sets it), and the largest gap (log2 units) between the
+// running maximum and a group's own maximum that the group's weights are
+// scaled up by.
+constexpr int kMaxFixedExp = 100;
+constexpr float kMaxGroupGap = 60.f;
 
-// Per-lane running state of one warp's online softmax.
-template <int CW>
+// Per-lane running state of one warp's online softmax.  m is warp-uniform
+// (log2 units); l and beta cover the token this lane owns in every group;
+// facc holds the lane's value column (4 channels over every token of the
+// warp's groups) in fp32.  Quantised cells carry each group's value weights
+// in 16-bit fixed point, round(w * 2^d * scale * sF) with sF = kMult * 2^F
+// warp-uniform and d the group's own gap below the running maximum, and add
+// the group's exact integer column sums into facc.
+template <int D>
 struct WarpState {
-  float m, l, beta;
-  float2 acc[CW / 2];
+  float m, l;
+  float beta[D / kGroup];
+  float facc[4];
+  float sF, slim;  // scale of w * scale, and the largest value scale it admits (w <= 1)
+  int F;
 };
 
 // Slot (in floats) of the 16-byte piece v (channels CW*k + 4v .. +3) in a
@@ -306,13 +311,13 @@ __device__ __forceinline__ int q2_slot(int k, int v) { return v * 16 + ((k + v) 
 // unfinished key group: keys from the exact residual, tokens past the end
 // masked.
 template <int KIND, int D, bool FULLV, bool TAIL>
-__device__ __forceinline__ void group_step(const uint8_t* st, const float* qconst, float* q2buf,
+__device__ __forceinline__ void group_step(const uint8_t* st, const float* qconst, float* q2buf, uint8_t* vbuf,
                                            const float* qfr, const __nv_bfloat16* res, int tok0, int nn,
-                                           int lane, int r, int k, float* logits_g,
-                                           WarpState<Cfg<KIND, D, FULLV>::kCW>& ws) {
+                                           int lane, int r, int k, float* logits_g, WarpState<D>& ws) {
   using C = Cfg<KIND, D, FULLV>;
   using R = typename C::R;
   constexpr int CH = C::kCH, CW = C::kCW, NWRD = C::kNWRD, TS = C::kTS, TPL = C::kTPL, HALF = C::kHalf;
+  constexpr int VG = C::kVG, COLS = C::kCols, LPC = C::kLPC;
   const float esc = pow2i(C::kE);
 
   // this lane's plane words of token j: rowbase + a compile-time offset
@@ -425,83 +430,155 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
       part[j] = s2.x + s2.y;
     }
   }
-  // all-reduce each token's logit over its CH lanes
-#pragma unroll
-  for (int j = 0; j < TPL; ++j)
-#pragma unroll
-    for (int o = 1; o < CH; o <<= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+  // ---- the logit of this lane's token tk = r + 8k: a transposed all-reduce
+  //      over the 4 lanes of token row r, after which each lane keeps one
+  //      token (k selects j = k among the row's tokens r + 8j)
+  static_assert(CH == 4 && TPL == 4, "the transposed reduction assumes 4 lanes and 4 tokens per lane");
+  float L;
+  {
+    const bool up = k & 2;
+    const float s0 = up ? part[0] : part[2], s1 = up ? part[1] : part[3];
+    const float k0 = up ? part[2] : part[0], k1 = up ? part[3] : part[1];
+    const float q0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 2);
+    const float q1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 2);
+    const bool odd = k & 1;
+    L = (odd ? q1 : q0) + __shfl_xor_sync(0xffffffffu, odd ? q0 : q1, 1);
+  }
+  const int tk = r + TS * k;
+  const bool valid = !TAIL || tok0 + tk < nn;
+  L = valid ? L * esc : -INFINITY;
+  // every lane's coefficient reads are done before the buffer takes weights
+  // (the shuffles above do not order shared-memory accesses)
+  __syncwarp();
 
   // ---- online softmax over the group (log2 units)
-  float gm = -INFINITY;
+  float gm = L;
 #pragma unroll
-  for (int j = 0; j < TPL; ++j)
-    if (!TAIL || tok0 + r + TS * j < nn) gm = fmaxf(gm, part[j]);
-#pragma unroll
-  for (int o = CH; o < 32; o <<= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
-  gm *= esc;
+  for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
   if (gm > ws.m) {
-    const float c = fast_exp2(ws.m - gm);
+    const float c = fast_exp2(ws.m - gm);  // 0 before the first group
     ws.l *= c;
-    ws.beta *= c;
 #pragma unroll
-    for (int i = 0; i < CW / 2; ++i) ws.acc[i] = __fmul2_rn(ws.acc[i], make_float2(c, c));
+    for (int g = 0; g < VG; ++g) ws.beta[g] *= c;
+#pragma unroll
+    for (int f = 0; f < 4; ++f) ws.facc[f] *= c;
     ws.m = gm;
   }
-  // weights carry 2^kVSh (undone once at the end)
-  const float off = static_cast<float>(C::kVSh) - ws.m;
-  float wgt[TPL];
-#pragma unroll
-  for (int j = 0; j < TPL; ++j) {
-    wgt[j] = fast_exp2(fmaf(part[j], esc, off));
-    if (TAIL && tok0 + r + TS * j >= nn) wgt[j] = 0.f;
-    ws.l += wgt[j];
-  }
-  if constexpr (C::kLogits) {
-    float mine = part[0];
-#pragma unroll
-    for (int j = 1; j < TPL; ++j) mine = (j == k) ? part[j] : mine;
-    logits_g[r + TS * k] = mine * esc;
-  }
+  // the group's own gap d below the running maximum (an integer, warp-
+  // uniform): its weights are scaled by 2^d so that its largest is in (1/2, 1]
+  const float dref = C::kQuant ? floorf(fminf(ws.m - gm, kMaxGroupGap)) : 0.f;
+  const float pw = pow2i(-static_cast<int>(dref));
+  const float wg = valid ? fast_exp2(L - ws.m + dref) : 0.f;
+  const float w = wg * pw;
+  ws.l += w;
+  if constexpr (C::kLogits) logits_g[tk] = L;
 
-  // ---- values
-#pragma unroll
-  for (int j = 0; j < TPL; ++j) {
-    if constexpr (C::kQuant) {
-      const uint32_t mv = *reinterpret_cast<const uint32_t*>(
-          st + ((TS * j) >> 4) * HALF + R::kVMetaOff +
-          ((r + ((TS * j) & 15)) * (D / kGroup) + (CW * k) / kGroup) * 4);
-      float s = bf16_lo(mv), mn = bf16_hi(mv);
-      if (TAIL && tok0 + r + TS * j >= nn) s = mn = 0.f;
-      uint32_t vh[NWRD], vl[NWRD];
-      plane_words(j, R::kVHi, vh);
-      const float wsc = wgt[j] * s;
-      if constexpr (C::kFourV) {
-        const float2 ww = make_float2(wsc, wsc);
-        plane_words(j, R::kQ4VLo, vl);
-        ws.beta = fmaf(wgt[j], mn, ws.beta);
-#pragma unroll
-        for (int u = 0; u < NWRD; ++u) axpy16<true>(ws.acc + 8 * u, ww, vh[u], vl[u]);
-      } else {
-        // 4-bit high plane: the weight carries the factor 4 of 4*hi
-        const uint32_t wh = __half_as_ushort(__float2half_rn(C::kQ4 ? 4.f * wsc : wsc));
-        ws.beta = fmaf(wgt[j], C::kQ4 ? fmaf(1.5f, s, mn) : mn, ws.beta);
-#pragma unroll
-        for (int u = 0; u < NWRD; ++u) axpy16_h(ws.acc + 8 * u, wh, vh[u]);
-      }
+  // ---- values: the owner of token tk turns its weight into per-group value
+  //      weights; then every lane runs its column over all 32 tokens
+  const int ob = tk >> 4, orow = tk & 15;
+  const int col = lane % COLS, hb = lane / COLS;
+  if constexpr (C::kQuant) {
+    const uint8_t* mp = st + ob * HALF + R::kVMetaOff + orow * (VG * 4);
+    uint32_t mv[VG];
+    if constexpr (VG == 4) {
+      const uint4 x = *reinterpret_cast<const uint4*>(mp);
+      mv[0] = x.x;
+      mv[1] = x.y;
+      mv[2] = x.z;
+      mv[3] = x.w;
     } else {
-      const uint4* vp = reinterpret_cast<const uint4*>(st + ((TS * j) >> 4) * HALF + R::kBfV +
-                                                       (r + ((TS * j) & 15)) * D * 2 + 2 * CW * k);
-      const float2 ww = make_float2(wgt[j], wgt[j]);
-      // past the end of the tail group the stage holds stale bytes, which
-      // may read as Inf / NaN: skip them rather than multiply by zero
-      if (TAIL && tok0 + r + TS * j >= nn) continue;
+      const uint2 x = *reinterpret_cast<const uint2*>(mp);
+      mv[0] = x.x;
+      mv[1] = x.y;
+    }
+    float sv[VG];
+    float smax = 0.f;
 #pragma unroll
-      for (int v = 0; v < CW / 8; ++v) {
-        const uint4 a = vp[v];
-        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+    for (int g = 0; g < VG; ++g) {
+      const float sc = bf16_lo(mv[g]), mn = bf16_hi(mv[g]);
+      sv[g] = valid ? sc : 0.f;
+      smax = fmaxf(smax, sv[g]);
+      // the minimum (plus the bucket midpoint of the high plane) of every
+      // channel of the group, weighted once per token
+      const float base = C::kLogits ? fmaf(1.5f, sc, mn) : mn;
+      if (valid) ws.beta[g] = fmaf(w, base, ws.beta[g]);
+    }
+    // fixed-point scale: every 2^d w * scale * sF stays below 2^15 (2^d w
+    // <= 1); a larger scale than any seen so far lowers F for the whole warp
+    if (__any_sync(0xffffffffu, smax >= ws.slim)) {
+      float x = smax;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+      const int e = min(static_cast<int>((__float_as_uint(x * C::kMult) >> 23) & 0xFFu) - 127, kMaxFixedExp + 14);
+      ws.F = min(14 - e, kMaxFixedExp);
+      ws.sF = C::kMult * pow2i(ws.F);
+      ws.slim = pow2i(15 - ws.F) / C::kMult;
+    }
+    const float wF = wg * ws.sF;
+    uint16_t* av = reinterpret_cast<uint16_t*>(vbuf);
+#pragma unroll
+    for (int g = 0; g < VG; ++g) {
+      av[g * 32 + tk] = static_cast<uint16_t>(round_fixed(wF, sv[g]));
+      if constexpr (C::kFourV) av[(VG + g) * 32 + tk] = static_cast<uint16_t>(round_fixed(0.25f * wF, sv[g]));
+    }
+    __syncwarp();
+    // this lane's column: the weight pairs of its value group, token order;
+    // exact integer sums of the group (below 2^24), then added in fp32
+    const uint32_t* ap = reinterpret_cast<const uint32_t*>(vbuf) + ((4 * col) / kGroup) * 16;
+    uint32_t acc[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int bi = 0; bi < 2 / LPC; ++bi) {
+      const int blk = LPC == 1 ? bi : hb;
+      const uint4 cw = *reinterpret_cast<const uint4*>(st + blk * HALF + R::kVHi + col * 16);
+      const uint4 a0 = *reinterpret_cast<const uint4*>(ap + 8 * blk);
+      const uint4 a1 = *reinterpret_cast<const uint4*>(ap + 8 * blk + 4);
+      column_dot(acc, cw.x, a0.x, a0.y);
+      column_dot(acc, cw.y, a0.z, a0.w);
+      column_dot(acc, cw.z, a1.x, a1.y);
+      column_dot(acc, cw.w, a1.z, a1.w);
+      if constexpr (C::kFourV) {
+        // the low plane is row-major: gather byte col of every token row
+        const uint8_t* lp = st + blk * HALF + R::kQ4VLo + col;
+        const uint32_t* apl = ap + VG * 16;
+        uint32_t lw[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          ws.acc[4 * v + i] = __ffma2_rn(ww, make_float2(bf16_lo(w[i]), bf16_hi(w[i])), ws.acc[4 * v + i]);
+          lw[i] = static_cast<uint32_t>(lp[(4 * i) * R::kRow]) | (static_cast<uint32_t>(lp[(4 * i + 1) * R::kRow]) << 8) |
+                  (static_cast<uint32_t>(lp[(4 * i + 2) * R::kRow]) << 16) |
+                  (static_cast<uint32_t>(lp[(4 * i + 3) * R::kRow]) << 24);
+        const uint4 l0 = *reinterpret_cast<const uint4*>(apl + 8 * blk);
+        const uint4 l1 = *reinterpret_cast<const uint4*>(apl + 8 * blk + 4);
+        column_dot(acc, lw[0], l0.x, l0.y);
+        column_dot(acc, lw[1], l0.z, l0.w);
+        column_dot(acc, lw[2], l1.x, l1.y);
+        column_dot(acc, lw[3], l1.z, l1.w);
+      }
+    }
+    // back to value units: 2^-(F + d), and 1/4 for the odd fields
+    const float u0 = pow2i(-ws.F) * pw, u1 = 0.25f * u0;
+#pragma unroll
+    for (int f = 0; f < 4; ++f) ws.facc[f] = fmaf(__uint2float_rn(acc[f]), (f & 1) ? u1 : u0, ws.facc[f]);
+  } else {
+    float* wv = reinterpret_cast<float*>(vbuf);
+    wv[tk] = w;
+    __syncwarp();
+#pragma unroll
+    for (int bi = 0; bi < 2 / LPC; ++bi) {
+      const int blk = LPC == 1 ? bi : hb;
+#pragma unroll 4
+      for (int t = 0; t < kBlock; ++t) {
+        // past the end of the tail group the stage holds stale bytes, which
+        // may read as Inf / NaN: skip them rather than multiply by zero
+        if (TAIL && tok0 + kBlock * blk + t >= nn) break;
+        const uint2 x = *reinterpret_cast<const uint2*>(st + blk * HALF + R::kBfV + t * D * 2 + col * 8);
+        const float wt = wv[kBlock * blk + t];
+        const float2 ww = make_float2(wt, wt);
+        float2 a01 = __ffma2_rn(ww, make_float2(bf16_lo(x.x), bf16_hi(x.x)), make_float2(ws.facc[0], ws.facc[1]));
+        float2 a23 = __ffma2_rn(ww, make_float2(bf16_lo(x.y), bf16_hi(x.y)), make_float2(ws.facc[2], ws.facc[3]));
+        ws.facc[0] = a01.x;
+        ws.facc[1] = a01.y;
+        ws.facc[2] = a23.x;
+        ws.facc[3] = a23.y;
       }
     }
   }
@@ -515,14 +592,15 @@ template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB, bool GQ>
 __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodeParams p) {
   using C = Cfg<KIND, D, FULLV>;
   using R = typename C::R;
-  constexpr int CH = C::kCH, CW = C::kCW, NSW = C::kNSW, TS = C::kTS;
+  constexpr int CH = C::kCH, NSW = C::kNSW;
   constexpr int LOAD = C::kLoad, STAGE = C::kStage;
+  constexpr int COLS = C::kCols, LPC = C::kLPC, VG = C::kVG;
 
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem sp = smem_plan(STAGE, NSW, p.chunk_groups, D, C::kLogits);
   float* logits = reinterpret_cast<float*>(smem + sp.logits);
-  auto wscr_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w); };
-  constexpr int kCorrOff = TS * D * 4;  // after the warp's TS x D partial sums
+  auto wres_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w); };
+  constexpr int kCorrOff = D * 4;  // after the warp's D channel sums
   auto corr_of = [&](int w) { return reinterpret_cast<float*>(smem + sp.rings + sp.ring_bytes * w + kCorrOff); };
   // the CTA's per-channel sums in its own scale, after warp 0's corrections
   float* cacc = reinterpret_cast<float*>(smem + sp.rings + kCorrOff + D * 4);
@@ -599,12 +677,16 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   if constexpr (CLUSTER) cluster_arrive_relaxed();
 
   const int k = lane % CH, r = lane / CH;
-  WarpState<CW> ws;
+  WarpState<D> ws;
   ws.m = -INFINITY;
   ws.l = 0.f;
-  ws.beta = 0.f;
 #pragma unroll
-  for (int i = 0; i < CW / 2; ++i) ws.acc[i] = make_float2(0.f, 0.f);
+  for (int g = 0; g < VG; ++g) ws.beta[g] = 0.f;
+#pragma unroll
+  for (int f = 0; f < 4; ++f) ws.facc[f] = 0.f;
+  ws.F = kMaxFixedExp;
+  ws.sF = C::kMult * pow2i(kMaxFixedExp);
+  ws.slim = pow2i(15 - kMaxFixedExp) / C::kMult;
 
   // groups of this warp: gi = warp + kNW * it
   const int nit = (!bad && cg > warp) ? (cg - warp + kNW - 1) / kNW : 0;
@@ -678,6 +760,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     // for the subnormal code views; both in shared memory for all warps
     float* qconst = reinterpret_cast<float*>(smem + sp.qconst);
     float* q2buf = reinterpret_cast<float*>(smem + sp.q2buf) + warp * 128;
+    uint8_t* vbuf = reinterpret_cast<uint8_t*>(q2buf);  // the same 512 B, reused after the keys
     for (int c = lane; c < D; c += 32) {
       const float qv = __bfloat162float(p.q[(static_cast<size_t>(b) * p.H + blockIdx.y) * D + c]) * p.sm_scale_log2;
       const int i = c & 15;
@@ -687,10 +770,10 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     }
     __syncwarp();
     // bf16 cells keep this lane's query channels in registers
-    float qfr[C::kQuant ? 1 : CW];
+    float qfr[C::kQuant ? 1 : C::kCW];
     if constexpr (!C::kQuant) {
 #pragma unroll
-      for (int i = 0; i < CW; ++i) qfr[i] = qconst[CW * k + i];
+      for (int i = 0; i < C::kCW; ++i) qfr[i] = qconst[C::kCW * k + i];
     }
     const __nv_bfloat16* res = C::kQuant ? p.residual + (static_cast<size_t>(b) * Hkv + hk) * kGroup * D : nullptr;
 
@@ -708,9 +791,9 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       const uint8_t* st = ring + stage * STAGE;
       float* lg = logits + gi * kGroup;
       if (tok0 + kGroup <= nn)
-        group_step<KIND, D, FULLV, false>(st, qconst, q2buf, qfr, res, tok0, nn, lane, r, k, lg, ws);
+        group_step<KIND, D, FULLV, false>(st, qconst, q2buf, vbuf, qfr, res, tok0, nn, lane, r, k, lg, ws);
       else
-        group_step<KIND, D, FULLV, true>(st, qconst, q2buf, qfr, res, tok0, nn, lane, r, k, lg, ws);
+        group_step<KIND, D, FULLV, true>(st, qconst, q2buf, vbuf, qfr, res, tok0, nn, lane, r, k, lg, ws);
       // every shared-memory read of this stage has been consumed above, so
       // the stage can be refilled
       __syncwarp();
@@ -720,43 +803,65 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   pdl_wait_prior_grid();  // nothing below may run ahead of the previous kernel
   if (!p.pdl_early) pdl_allow_dependents();
 
-  // ---- this warp's result in its own scale 2^-m_w: true per-channel sums,
-  //      reduced over the token sub-groups
+  const int h = GQ ? cta_id_y() : hk;  // query head
+
+  // ---- this warp's result in its own scale 2^-m_w: true per-channel sums
+  //      (lane (hb, col) holds channels 4 col .. 4 col + 3)
   float lw;
   {
-    const float unsh = pow2i(-C::kVSh);
-    float o[CW];
+    lw = ws.l;
 #pragma unroll
-    for (int i = 0; i < CW / 2; ++i) {
-      if constexpr (C::kHalfV) {
-        // pair i of word u: channels 16u + (i & 7) and 16u + (i & 7) + 8
-        const int u = i >> 3, ii = i & 7;
-        const float sc = pow2i(24 - posh(ii) - C::kVSh);
-        o[16 * u + ii] = fmaf(ws.acc[i].x, sc, ws.beta * unsh);
-        o[16 * u + ii + 8] = fmaf(ws.acc[i].y, sc, ws.beta * unsh);
-      } else if constexpr (C::kQuant) {
-        const int pa = pos4((2 * i) & 15);
-        const int pb = pos4((2 * i + 1) & 15);
-        o[2 * i] = fmaf(ws.acc[i].x, pow2i(64 - pa), ws.beta * unsh);
-        o[2 * i + 1] = fmaf(ws.acc[i].y, pow2i(64 - pb), ws.beta * unsh);
-      } else {
-        o[2 * i] = ws.acc[i].x;
-        o[2 * i + 1] = ws.acc[i].y;
+    for (int off = 16; off > 0; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+    const int col = lane % COLS, hb = lane / COLS, gv = (4 * col) / kGroup;
+    float o[4];
+    if constexpr (C::kQuant) {
+      // the value minima of the lane's group, summed over the owned tokens
+      float bsum[VG];
+#pragma unroll
+      for (int g = 0; g < VG; ++g) {
+        bsum[g] = ws.beta[g];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) bsum[g] += __shfl_xor_sync(0xffffffffu, bsum[g], off);
+      }
+      float bmine = bsum[0];
+#pragma unroll
+      for (int g = 1; g < VG; ++g) bmine = gv == g ? bsum[g] : bmine;
+#pragma unroll
+      for (int f = 0; f < 4; ++f) o[f] = ws.facc[f];
+      if constexpr (LPC == 2) {
+#pragma unroll
+        for (int f = 0; f < 4; ++f) o[f] += __shfl_xor_sync(0xffffffffu, o[f], 16);
+      }
+#pragma unroll
+      for (int f = 0; f < 4; ++f) o[f] += bmine;
+    } else {
+#pragma unroll
+      for (int f = 0; f < 4; ++f) o[f] = ws.facc[f];
+      if constexpr (LPC == 2) {
+#pragma unroll
+        for (int f = 0; f < 4; ++f) o[f] += __shfl_xor_sync(0xffffffffu, o[f], 16);
       }
     }
-    lw = ws.l * unsh;
+    // the current token of the cell's own loop (exact K and V, one more
+    // softmax entry after the stored tokens): warp 0 of the last split
+    if (p.k_cur != nullptr && split == S - 1 && warp == 0 && !cta_i[kSlotBad]) {
+      const size_t kv_row = (static_cast<size_t>(b) * Hkv + hk) * D;
+      const __nv_bfloat16* qh = p.q + (static_cast<size_t>(b) * p.H + h) * D;
+      float sd = 0.f;
+      for (int c = lane; c < D; c += 32)
+        sd = fmaf(__bfloat162float(qh[c]) * p.sm_scale_log2, __bfloat162float(p.k_cur[kv_row + c]), sd);
 #pragma unroll
-    for (int off = CH; off < 32; off <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
-    // every lane stores its partial sums; the combine adds the TS token
-    // sub-groups (16-byte pieces rotated so that each store is conflict-free)
-    float* wsc = wscr_of(warp) + r * D + k * CW;
+      for (int off = 16; off > 0; off >>= 1) sd += __shfl_xor_sync(0xffffffffu, sd, off);
+      const float mnew = fmaxf(ws.m, sd);
+      const float a = fast_exp2(ws.m - mnew), bw = fast_exp2(sd - mnew);
+      lw = fmaf(lw, a, bw);
 #pragma unroll
-    for (int v = 0; v < CW / 4; ++v)
-      *reinterpret_cast<float4*>(wsc + 4 * wscr_piece<CW>(v, k, r)) =
-          make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+      for (int f = 0; f < 4; ++f) o[f] = fmaf(o[f], a, bw * __bfloat162float(p.v_cur[kv_row + 4 * col + f]));
+      ws.m = mnew;
+    }
+    if (hb == 0) *reinterpret_cast<float4*>(wres_of(warp) + 4 * col) = make_float4(o[0], o[1], o[2], o[3]);
   }
 
-  const int h = GQ ? cta_id_y() : hk;  // query head
   const int HC = head_cl ? 1 << p.g_log2 : 1;
   const int rbase = S * (h & (HC - 1));  // cluster rank of this head's split 0
 
@@ -780,18 +885,11 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
 #pragma unroll
   for (int w = 0; w < kNW; ++w) m_c = fmaxf(m_c, table[split * kNW + w].x);
   for (int c = threadIdx.x; c < D; c += kThreads) {
-    const int kc = c / CW, i = c % CW;
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < kNW; ++w) {
       const float mw = table[split * kNW + w].x;
-      if (mw != -INFINITY) {
-        const float* wsc = wscr_of(w) + kc * CW + (i & 3);
-        float sw = 0.f;
-#pragma unroll
-        for (int rr = 0; rr < TS; ++rr) sw += wsc[rr * D + 4 * wscr_piece<CW>(i >> 2, kc, rr)];
-        v = fmaf(fast_exp2(mw - m_c), sw, v);
-      }
+      if (mw != -INFINITY) v = fmaf(fast_exp2(mw - m_c), wres_of(w)[c], v);
     }
     cacc[c] = v;
   }
@@ -1012,37 +1110,87 @@ size_t smem_bytes_t(int cg) {
   return smem_plan(C::kStage, C::kNSW, cg, D, C::kLogits).total;
 }
 
-// CTAs of this instantiation that can be resident at once on the device
-// (for clusters of splits x hc: co-resident clusters times the cluster size).
-template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB, bool GQ = false>
-long resident_ctas_t(int cg, int splits, int hc, int sms) {
-  const size_t smem = smem_bytes_t<KIND, D, FULLV>(cg);
-  if (smem > 227u * 1024u) return 0;
+// Host-side launch state, set up once per (kernel build, device) and shared
+// by every thread: the dynamic shared-memory limit of each build is raised
+// once to the largest size a CTA may request (so no call ever lowers it
+// under another thread's launch), non-portable cluster sizes are allowed
+// once, and the device's SM count and every occupancy answer are cached.
+constexpr int kMaxDevices = 64;
+
+int device_sms(int* dev_out) {
+  static std::mutex mu;
+  static int sms_of[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = -1;
+  if (dev_out) *dev_out = dev;
+  if (dev < 0) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (sms_of[dev] == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 148;
+    sms_of[dev] = sms;
+  }
+  return sms_of[dev];
+}
+
+template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB, bool GQ>
+cudaError_t prepare_kernel(int dev) {
+  static std::mutex mu;
+  static bool done[kMaxDevices] = {};
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev]) return cudaSuccess;
   auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-    return 0;
-  if (CLUSTER && splits * hc > 8 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-    return 0;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kMaxDynamicSmem));
+  if (e == cudaSuccess && CLUSTER) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) done[dev] = true;
+  return e;
+}
+
+// CTAs of this instantiation that can be resident at once on the device
+// (for clusters of splits x hc: co-resident clusters times the cluster size);
+// 0 when the build cannot run the configuration.  Answers are cached.
+template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB, bool GQ = false>
+long resident_ctas_t(int cg, int splits, int hc) {
+  const size_t smem = smem_bytes_t<KIND, D, FULLV>(cg);
+  if (smem > kMaxDynamicSmem) return 0;
+  int dev = -1;
+  const int sms = device_sms(&dev);
+  if (dev < 0 || prepare_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>(dev) != cudaSuccess) return 0;
+  static std::mutex mu;
+  static std::map<std::tuple<int, size_t, int, int>, long> cache;
+  const auto key = std::make_tuple(dev, smem, splits, hc);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>;
+  long slots = 0;
   if (!CLUSTER) {
     int blocks = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kThreads, smem) != cudaSuccess) return 0;
-    return static_cast<long>(blocks) * sms;
+    slots = static_cast<long>(blocks) * sms;
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(splits, hc, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = splits;
+    attr.val.clusterDim.y = hc;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return 0;
+    slots = static_cast<long>(clusters) * splits * hc;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(splits, hc, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = splits;
-  attr.val.clusterDim.y = hc;
-  attr.val.clusterDim.z = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return 0;
-  return static_cast<long>(clusters) * splits * hc;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = slots;
+  return slots;
 }
 
 // balance: ask the hardware to place a cluster's CTAs on the least loaded
@@ -1051,14 +1199,12 @@ template <int KIND, int D, bool FULLV, bool CLUSTER, int MINB, bool GQ>
 cudaError_t launch_t(const DecodeParams& p, int batch, int splits, int hc, cudaStream_t stream, bool pdl,
                      bool balance) {
   const size_t smem = smem_bytes_t<KIND, D, FULLV>(p.chunk_groups);
-  if (smem > 227u * 1024u) return cudaErrorInvalidValue;
+  if (smem > kMaxDynamicSmem) return cudaErrorInvalidValue;
   auto kern = decode_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  int dev = -1;
+  device_sms(&dev);
+  cudaError_t e = prepare_kernel<KIND, D, FULLV, CLUSTER, MINB, GQ>(dev);
   if (e != cudaSuccess) return e;
-  if (CLUSTER && splits * hc > 8) {  // grouped queries: up to 16 CTAs per cluster
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(splits, p.H, batch);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1089,9 +1235,9 @@ cudaError_t launch_t(const DecodeParams& p, int batch, int splits, int hc, cudaS
 }
 
 template <int KIND, int D, bool FULLV, int MINB>
-long resident_m(int cg, int splits, int hc, int sms) {
-  return splits * hc > 1 ? resident_ctas_t<KIND, D, FULLV, true, MINB>(cg, splits, hc, sms)
-                         : resident_ctas_t<KIND, D, FULLV, false, MINB>(cg, splits, 1, sms);
+long resident_m(int cg, int splits, int hc) {
+  return splits * hc > 1 ? resident_ctas_t<KIND, D, FULLV, true, MINB>(cg, splits, hc)
+                         : resident_ctas_t<KIND, D, FULLV, false, MINB>(cg, splits, 1);
 }
 
 // A grid of at least this many waves of 4-per-SM residency runs the
@@ -1107,13 +1253,11 @@ constexpr long kBalancedWaves = 2;
 
 template <int KIND, int D, bool FULLV>
 cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t stream, bool pdl) {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int hc = head_cluster(KIND, 1 << p.g_log2, FULLV);
   if (splits > kMaxClusterSplits || splits * hc > kMaxClusterCtas) return cudaErrorInvalidValue;
   const bool cl = splits * hc > 1;
   const long ctas = static_cast<long>(batch) * p.H * splits;
-  const long slots4 = resident_m<KIND, D, FULLV, 4>(p.chunk_groups, splits, hc, sms);
+  const long slots4 = resident_m<KIND, D, FULLV, 4>(p.chunk_groups, splits, hc);
   const bool balance = cl && slots4 > 0 && ctas <= kBalancedWaves * slots4;
   DecodeParams q = p;
   q.pdl_early = slots4 <= 0 || ctas > slots4;
@@ -1123,7 +1267,7 @@ cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t 
               : launch_t<KIND, D, FULLV, false, 4, true>(q, batch, splits, 1, stream, pdl, false);
   if constexpr (KIND != LOOPKV_CELL_BF16 && !FULLV) {
     if (slots4 > 0 && ctas >= kHighOccupancyWaves * slots4 &&
-        resident_m<KIND, D, FULLV, 5>(p.chunk_groups, splits, 1, sms) > slots4)
+        resident_m<KIND, D, FULLV, 5>(p.chunk_groups, splits, 1) > slots4)
       return cl ? launch_t<KIND, D, FULLV, true, 5, false>(q, batch, splits, 1, stream, pdl, balance)
                 : launch_t<KIND, D, FULLV, false, 5, false>(q, batch, splits, 1, stream, pdl, false);
   }
@@ -1133,23 +1277,23 @@ cudaError_t launch_c(const DecodeParams& p, int batch, int splits, cudaStream_t 
 
 // Co-resident CTAs of one decode build (0 without a device); minb 5 only
 // exists for the 4-bit and 2-bit kinds.
-long resident_ctas(int kind, int d, int cg, int splits, int hc, int sms, int minb) {
+long resident_ctas(int kind, int d, int cg, int splits, int hc, int minb) {
   if (minb == 5) {
     switch (kind * 1000 + d) {
-      case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 5>(cg, splits, hc, sms);
-      case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 5>(cg, splits, hc, sms);
-      case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 5>(cg, splits, 1, sms);
-      case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 5>(cg, splits, 1, sms);
+      case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 5>(cg, splits, hc);
+      case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 5>(cg, splits, hc);
+      case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 5>(cg, splits, 1);
+      case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 5>(cg, splits, 1);
       default: return 0;
     }
   }
   switch (kind * 1000 + d) {
-    case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 4>(cg, splits, hc, sms);
-    case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 4>(cg, splits, hc, sms);
-    case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 4>(cg, splits, 1, sms);
-    case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 4>(cg, splits, 1, sms);
-    case LOOPKV_CELL_BF16 * 1000 + 128: return resident_m<LOOPKV_CELL_BF16, 128, false, 4>(cg, splits, 1, sms);
-    case LOOPKV_CELL_BF16 * 1000 + 64: return resident_m<LOOPKV_CELL_BF16, 64, false, 4>(cg, splits, 1, sms);
+    case LOOPKV_CELL_Q4 * 1000 + 128: return resident_m<LOOPKV_CELL_Q4, 128, false, 4>(cg, splits, hc);
+    case LOOPKV_CELL_Q4 * 1000 + 64: return resident_m<LOOPKV_CELL_Q4, 64, false, 4>(cg, splits, hc);
+    case LOOPKV_CELL_Q2 * 1000 + 128: return resident_m<LOOPKV_CELL_Q2, 128, false, 4>(cg, splits, 1);
+    case LOOPKV_CELL_Q2 * 1000 + 64: return resident_m<LOOPKV_CELL_Q2, 64, false, 4>(cg, splits, 1);
+    case LOOPKV_CELL_BF16 * 1000 + 128: return resident_m<LOOPKV_CELL_BF16, 128, false, 4>(cg, splits, 1);
+    case LOOPKV_CELL_BF16 * 1000 + 64: return resident_m<LOOPKV_CELL_BF16, 64, false, 4>(cg, splits, 1);
     default: return 0;
   }
 }
@@ -1168,13 +1312,12 @@ int decode_splits(int kind, int head_dim, int batch, int heads, int max_seq_len,
   int s = 1;
   while (s < smax && (groups + s - 1) / s > kTargetGroupsPerSplit) s <<= 1;
   if (pairs <= 0 || groups <= 1) return s;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sms(nullptr);
   // ... and, past that, doubled while the grid fills less than 80 % of the
   // resident slots once (short grids: more, shorter CTAs put every SM to
   // work), keeping at least two groups per warp
   while (s < smax && groups >= 2 * kNW * 2 * s) {
-    long slots = resident_ctas(kind, head_dim, (groups + s - 1) / s, s, hc, sms, 4);
+    long slots = resident_ctas(kind, head_dim, (groups + s - 1) / s, s, hc, 4);
     if (slots <= 0) slots = 4L * sms;  // no device: a fixed guess keeps the choice deterministic
     if (pairs * s * 5 >= slots * 4) break;
     s <<= 1;

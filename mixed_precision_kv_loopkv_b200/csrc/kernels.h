@@ -45,6 +45,10 @@ struct DecodeParams {              // H = query heads, Hkv = KV heads
   const __nv_bfloat16* v_new;     // [B][1][Hkv][D]
   uint8_t* wr_arena;              // the same arena, writable
   __nv_bfloat16* wr_residual;     // the same key residual, writable
+  // optional current token (k_cur non-null): its exact key and value join
+  // the softmax after the seq_lens[b] stored tokens (no low plane)
+  const __nv_bfloat16* k_cur;     // [B][Hkv][D]
+  const __nv_bfloat16* v_cur;     // [B][Hkv][D]
 };
 
 cudaError_t launch_append(int kind, int head_dim, const AppendParams& p, int batch,

@@ -137,7 +137,8 @@ namespace {
 // split choice and launch.  k_new == nullptr: plain decode over seq_lens;
 // otherwise seq_lens holds start positions and the cell must be stored.
 loopkv_status decode_common(const loopkv_config* cfg, const loopkv_cells* cells, int32_t loop, int32_t layer,
-                            const void* k_new, const void* v_new, const void* q, const int32_t* block_table,
+                            const void* k_new, const void* v_new, const void* q, const void* k_cur,
+                            const void* v_cur, const int32_t* block_table,
                             const int32_t* seq_lens, int32_t batch, int32_t max_seq_len, float tau,
                             float sm_scale, void* out, uint32_t* sel_mask, int32_t* sel_count,
                             int32_t* err_flag, void* stream) {
@@ -166,6 +167,8 @@ loopkv_status decode_common(const loopkv_config* cfg, const loopkv_cells* cells,
   if (kind != LOOPKV_CELL_BF16 && (!residual || !aligned16(residual))) return LOOPKV_ERR_INVALID_ARG;
   if (!q || !aligned16(q) || !out || !block_table || !seq_lens) return LOOPKV_ERR_INVALID_ARG;
   if (fused && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return LOOPKV_ERR_INVALID_ARG;
+  // the current token: both rows or neither
+  if ((k_cur == nullptr) != (v_cur == nullptr)) return LOOPKV_ERR_INVALID_ARG;
   const int group = cfg->num_heads / kv_heads(cfg);  // query heads per KV head
   // grouped queries append through loopkv_quantize_append: in one launch the
   // other heads' CTAs would read the new token before its writer is done
@@ -208,6 +211,8 @@ loopkv_status decode_common(const loopkv_config* cfg, const loopkv_cells* cells,
   p.v_new = static_cast<const __nv_bfloat16*>(v_new);
   p.wr_arena = fused ? static_cast<uint8_t*>(arena) : nullptr;
   p.wr_residual = fused ? static_cast<__nv_bfloat16*>(residual) : nullptr;
+  p.k_cur = static_cast<const __nv_bfloat16*>(k_cur);
+  p.v_cur = static_cast<const __nv_bfloat16*>(v_cur);
   const cudaError_t e = loopkv::launch_decode(kind, cfg->head_dim, p, batch, splits, full_values,
                                               static_cast<cudaStream_t>(stream),
                                               (cfg->flags & LOOPKV_FLAG_PDL) != 0);
@@ -219,12 +224,12 @@ loopkv_status decode_common(const loopkv_config* cfg, const loopkv_cells* cells,
 extern "C" {
 
 loopkv_status loopkv_decode_attention(const loopkv_config* cfg, const loopkv_cells* cells,
-                                      int32_t loop, int32_t layer, const void* q,
-                                      const int32_t* block_table, const int32_t* seq_lens,
+                                      int32_t loop, int32_t layer, const void* q, const void* k_cur,
+                                      const void* v_cur, const int32_t* block_table, const int32_t* seq_lens,
                                       int32_t batch, int32_t max_seq_len, float tau,
                                       float sm_scale, void* out, uint32_t* sel_mask,
                                       int32_t* sel_count, int32_t* err_flag, void* stream) {
-  return decode_common(cfg, cells, loop, layer, nullptr, nullptr, q, block_table, seq_lens, batch,
+  return decode_common(cfg, cells, loop, layer, nullptr, nullptr, q, k_cur, v_cur, block_table, seq_lens, batch,
                        max_seq_len, tau, sm_scale, out, sel_mask, sel_count, err_flag, stream);
 }
 
@@ -236,7 +241,7 @@ loopkv_status loopkv_append_decode_attention(const loopkv_config* cfg, const loo
                                              float sm_scale, void* out, uint32_t* sel_mask,
                                              int32_t* sel_count, int32_t* err_flag, void* stream) {
   if (!k_new || !v_new) return LOOPKV_ERR_INVALID_ARG;
-  return decode_common(cfg, cells, loop, layer, k_new, v_new, q, block_table, start_pos, batch,
+  return decode_common(cfg, cells, loop, layer, k_new, v_new, q, nullptr, nullptr, block_table, start_pos, batch,
                        max_seq_len, tau, sm_scale, out, sel_mask, sel_count, err_flag, stream);
 }
 

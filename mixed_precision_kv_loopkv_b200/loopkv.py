@@ -58,8 +58,8 @@ def _load():
         "loopkv_residual_bytes": (ctypes.c_size_t, [P(loopkv_config)]),
         "loopkv_quantize_append": (ctypes.c_int, [P(loopkv_config), P(loopkv_cells), I32, I32, VP, VP,
                                                   VP, VP, I32, I32, VP, VP]),
-        "loopkv_decode_attention": (ctypes.c_int, [P(loopkv_config), P(loopkv_cells), I32, I32, VP, VP,
-                                                   VP, I32, I32, F32, F32, VP, VP, VP, VP, VP]),
+        "loopkv_decode_attention": (ctypes.c_int, [P(loopkv_config), P(loopkv_cells), I32, I32, VP, VP, VP,
+                                                   VP, VP, I32, I32, F32, F32, VP, VP, VP, VP, VP]),
         "loopkv_append_decode_attention": (ctypes.c_int, [P(loopkv_config), P(loopkv_cells), I32, I32, VP, VP,
                                                           VP, VP, VP, I32, I32, F32, F32, VP, VP, VP, VP,
                                                           VP]),
@@ -204,13 +204,16 @@ def loopkv_quantize_append(kv: KVCells, loop: int, layer: int, k_new, v_new, blo
 
 def loopkv_decode_attention(kv: KVCells, loop: int, layer: int, q, block_table, seq_lens, tau: float,
                             sm_scale: float = 1.0, out=None, max_seq_len: int = 0, sel_mask=None,
-                            sel_count=None, err_flag=None, stream=None):
-    """Decode attention of q bf16[B, H, D] over cell (loop, layer); returns out bf16[B, H, D]."""
+                            sel_count=None, err_flag=None, stream=None, k_cur=None, v_cur=None):
+    """Decode attention of q bf16[B, H, D] over cell (loop, layer); returns out bf16[B, H, D].
+    k_cur, v_cur (optional bf16 [B, Hkv, D] or [B, 1, Hkv, D]): the current
+    token's own K/V, attended exactly after the stored tokens."""
     if out is None:
         out = torch.empty_like(q)
     batch = int(q.shape[0])
     st = _lib.loopkv_decode_attention(
         ctypes.byref(kv.cfg), ctypes.byref(kv.cells), loop, layer, _ptr(q, "q", torch.bfloat16),
+        _ptr(k_cur, "k_cur", torch.bfloat16, optional=True), _ptr(v_cur, "v_cur", torch.bfloat16, optional=True),
         _ptr(block_table, "block_table", torch.int32), _ptr(seq_lens, "seq_lens", torch.int32),
         batch, int(max_seq_len), float(tau), float(sm_scale), _ptr(out, "out", torch.bfloat16),
         _ptr(sel_mask, "sel_mask", torch.int32, optional=True),

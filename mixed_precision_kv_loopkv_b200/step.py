@@ -9,7 +9,10 @@ position n:
   * a stored cell first appends the token's K/V at position n, then attends
     over n + 1 tokens;
   * a reuse cell of loop l < L-1 attends over the final loop's first n
-    tokens: the final loop has not produced this token's K/V yet.
+    tokens (the final loop has not produced this token's K/V yet) plus the
+    current token exactly as its own loop l computed it: the model projects
+    K/V in every loop, a reuse cell just stores none of them, so its own row
+    is passed to the kernel as one more, exact, token.
 The model's projections and MLPs are not part of this path; each cell's query
 and new K/V are given tensors.
 """
@@ -44,7 +47,10 @@ class LoopedDecodeStep:
     pos    : device int32[B], current length n of every sequence (the new
              token's position); ``advance()`` moves it by one on the device.
     q      : per cell, bf16[B, H, D]  (H query heads)
-    k_new, v_new : per stored cell, bf16[B, 1, Hkv, D] (None for reuse cells)
+    k_new, v_new : per cell, bf16[B, 1, Hkv, D]: the token's K/V as the cell's
+             loop computed it (appended by stored cells, attended exactly by
+             reuse cells; a reuse cell without an entry attends over the
+             stored tokens only)
     out    : per cell, bf16[B, H, D] (written)
     sel_count : optional per cell int32[B, H] (written)
     fused  : a stored cell runs append and attention as one launch
@@ -61,7 +67,8 @@ class LoopedDecodeStep:
         self.block_table = block_table
         self.pos = pos
         self.pos_next = pos + 1
-        self.q, self.k_new, self.v_new, self.out = q, k_new, v_new, out
+        self.q, self.out = q, out
+        self.k_new, self.v_new = dict(k_new), dict(v_new)
         self.tau, self.sm_scale, self.max_seq_len = tau, sm_scale, max_seq_len
         self.sel_count = sel_count
         self.err_flag = err_flag
@@ -92,10 +99,13 @@ class LoopedDecodeStep:
                 lens = self.pos_next
             else:
                 lens = self.pos
+            cur_k = cur_v = None
+            if kind == LOOPKV_CELL_REUSE and self.k_new.get(cell) is not None:
+                cur_k, cur_v = self.k_new[cell], self.v_new[cell]
             loopkv_decode_attention(kv, loop, layer, self.q[cell], self.block_table, lens, self.tau,
                                     self.sm_scale, out=self.out[cell], max_seq_len=self.max_seq_len,
                                     sel_count=None if self.sel_count is None else self.sel_count[cell],
-                                    err_flag=self.err_flag, stream=stream)
+                                    err_flag=self.err_flag, stream=stream, k_cur=cur_k, v_cur=cur_v)
 
     def advance(self):
         self.pos.add_(1)

@@ -79,10 +79,12 @@ def _cells(m, n):
 FAKE = ctypes.c_void_p(0x20000)
 
 
-def _decode(m, cfg, cells, loop=0, layer=0, tau=0.01, batch=1, max_seq_len=0, q=FAKE, sm_scale=1.0):
+def _decode(m, cfg, cells, loop=0, layer=0, tau=0.01, batch=1, max_seq_len=0, q=FAKE, sm_scale=1.0,
+            k_cur=None, v_cur=None):
     lib = m.library()
-    return lib.loopkv_decode_attention(ctypes.byref(cfg), ctypes.byref(cells), loop, layer, q, FAKE, FAKE,
-                                       batch, max_seq_len, tau, sm_scale, FAKE, None, None, None, None)
+    return lib.loopkv_decode_attention(ctypes.byref(cfg), ctypes.byref(cells), loop, layer, q, k_cur, v_cur,
+                                       FAKE, FAKE, batch, max_seq_len, tau, sm_scale, FAKE, None, None, None,
+                                       None)
 
 
 def _append(m, cfg, cells, loop=0, layer=0, batch=1, T=1, k=FAKE):
@@ -225,3 +227,13 @@ def test_grouped_query_split_cap(m):
     lib = m.library()
     assert lib.loopkv_decode_splits(ctypes.byref(big), Q4, 1, 16384) == 2
     assert lib.loopkv_decode_splits(ctypes.byref(big), Q4, 1, 65536) == 2
+
+
+def test_current_token_needs_both_rows(m):
+    """k_cur and v_cur come together: one without the other is an argument
+    error, reported before anything is launched."""
+    cfg = _cfg(m, [Q4, Q2, REUSE, Q4], 2, 2)
+    cfg.plan[2] = Q4
+    cells = _cells(m, 4)
+    assert _decode(m, cfg, cells, k_cur=FAKE) == 1
+    assert _decode(m, cfg, cells, v_cur=FAKE) == 1

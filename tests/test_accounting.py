@@ -44,3 +44,11 @@ def test_grouped_queries_count_the_cache_once_per_group():
     # one query per KV head: the per-head sum
     assert step_bytes(plan, 2, 1, 128, 2, lens, lens, [[[5, 7]] * 2, [[0, 0]] * 2]) == sum(
         decode_bytes(k, 128, n, s) for k, ss in (("q4", (5, 7)), ("q2", (0, 0))) for n in lens for s in ss)
+
+
+def test_reuse_current_token_adds_its_exact_row():
+    from mixed_precision_kv_loopkv_b200.accounting import step_bytes
+    plan = ["reuse", "q2", "q4", "q4"]
+    base = step_bytes(plan, 2, 2, 128, 2, [64], [64])
+    cur = step_bytes(plan, 2, 2, 128, 2, [64], [64], reuse_current=True)
+    assert cur - base == 2 * 4 * 128          # one reuse cell, two heads, K + V bf16 rows

@@ -57,8 +57,8 @@ def test_single_rank_helpers():
 def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "decode_attention_demo.md").write_text(
-        f"- source_sha256: `{bench.decode_source_hash()}`\n- dram_bytes_per_launch: 1234\n")
+    (prof / "decode_attention_demo.json").write_text(json.dumps(
+        {"source_sha256": bench.decode_source_hash(), "dram_bytes_per_launch": 1234}))
     csrc = tmp_path / "mixed_precision_kv_loopkv_b200" / "csrc"
     csrc.mkdir(parents=True)
     for f in ("decode.cu", "device_common.cuh"):
@@ -68,6 +68,39 @@ def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("demo") == 1234.0
     (csrc / "decode.cu").write_text("// changed\n")
     assert bench.profiled_traffic("demo") is None
+
+
+def test_ingest_ncu_weights_launches_by_plan(tmp_path, monkeypatch):
+    """The ncu launch log is parsed per source kind and weighted by the
+    plan's launches of each kind."""
+    from workload import get_workload, make_plan
+    hdr = ['"ID"', '"Kernel Name"', '"Metric Name"', '"Metric Value"']
+    lines = [",".join(hdr)]
+    vals = {("0", "q4"): (100.0, 1000.0), ("1", "q2"): (60.0, 600.0), ("2", "q4"): (300.0, 3000.0)}
+    for (lid, kind), (dram, inst) in vals.items():
+        t = {"q4": 0, "q2": 1}[kind]
+        name = f"void loopkv::decode_kernel<{t}, 128, 0, 1, 4, 0>(loopkv::DecodeParams)"
+        for metric, v in (("dram__bytes_read.sum", dram), ("dram__bytes_write.sum", 0.0),
+                          ("smsp__inst_executed.sum", inst), ("gpu__time_duration.sum", 5.0)):
+            lines.append(",".join(f'"{x}"' for x in (lid, name, metric, v)))
+    csv_path = tmp_path / "launches.csv"
+    csv_path.write_text("\n".join(lines) + "\n")
+    (tmp_path / "profiles").mkdir()
+    for f in ("decode.cu", "device_common.cuh"):
+        d = tmp_path / "mixed_precision_kv_loopkv_b200" / "csrc"
+        d.mkdir(parents=True, exist_ok=True)
+        (d / f).write_bytes(open(os.path.join(bench.ROOT, "mixed_precision_kv_loopkv_b200", "csrc", f), "rb").read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    out = bench.ingest_ncu(str(csv_path), "ouro_step", scale=2.0)
+    w = get_workload("ouro_step")
+    plan = make_plan(w)
+    L, N = w.num_loops, w.num_layers
+    src = [plan[c] if plan[c] != "reuse" else plan[(L - 1) * N + c % N] for c in range(len(plan))]
+    n4, n2 = src.count("q4"), src.count("q2")
+    assert out["per_kind"]["q4"]["dram_bytes_per_launch"] == 2 * 200.0
+    assert out["dram_bytes_per_launch"] == pytest.approx((n4 * 400.0 + n2 * 120.0) / (n4 + n2))
+    assert out["warp_instructions_per_launch"] == pytest.approx((n4 * 4000.0 + n2 * 1200.0) / (n4 + n2))
+    assert bench.profiled_traffic("ouro_step") == pytest.approx(out["dram_bytes_per_launch"])
 
 
 def test_sweep_overrides_and_strict_json():

@@ -122,15 +122,16 @@ def test_append_flags_bad_block_and_overflow():
     assert int(err) & LOOPKV_DEVERR_SEQ_LEN
 
 
-def test_append_flags_value_scale_out_of_range():
-    from mixed_precision_kv_loopkv_b200 import LOOPKV_DEVERR_RANGE, KVCells, loopkv_quantize_append
+def test_large_value_scales_need_no_flag():
+    """Value scales have no limit: a 32-channel range of 5000 (scale 333 at
+    4 bits) is stored without any device error."""
+    from mixed_precision_kv_loopkv_b200 import KVCells, loopkv_quantize_append
     kv = KVCells(["q4"], 1, 1, 1, 64, 2, 1, 2)
     table = torch.tensor([[0, 1]], dtype=torch.int32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     k = torch.randn(1, 4, 1, 64, device="cuda").to(torch.bfloat16)
     v = k.clone()
+    v[0, 3, 0, 7] = 5000.0
     loopkv_quantize_append(kv, 0, 0, k, v, table, torch.zeros(1, dtype=torch.int32, device="cuda"), err_flag=err)
+    torch.cuda.synchronize()
     assert int(err) == 0
-    v[0, 3, 0, 7] = 5000.0          # range 5000 / 15 > 255
-    loopkv_quantize_append(kv, 0, 0, k, v, table, torch.zeros(1, dtype=torch.int32, device="cuda"), err_flag=err)
-    assert int(err) & LOOPKV_DEVERR_RANGE
