@@ -87,28 +87,22 @@ __device__ __forceinline__ void combine_planes(uint32_t hi, uint32_t lo, uint32_
 }
 
 // Dot product of the subnormal code views of one 16-channel word with 8
-// coefficient pairs (channels 2p, 2p+1), two short chains.
+// coefficient pairs (channels 2p, 2p+1), accumulated into acc (one chain;
+// a lane interleaves the chains of its four tokens).
 template <bool FOUR>
-__device__ __forceinline__ float2 dot16(const float2* c, uint32_t a, uint32_t b, float2 acc0) {
-  float2 acc1 = make_float2(0.f, 0.f);
+__device__ __forceinline__ float2 dot16(const float2* c, uint32_t a, uint32_t b, float2 acc) {
   if constexpr (FOUR) {  // a, b = high / low plane words
     uint32_t e, o;
     combine_planes(a, b, e, o);
     const uint32_t e20 = e >> 20, o20 = o >> 20;
 #pragma unroll
-    for (int m = 0; m < 8; m += 2) {
-      acc0 = __ffma2_rn(c[m], make_float2(nib(e, e20, m), nib(o, o20, m)), acc0);
-      acc1 = __ffma2_rn(c[m + 1], make_float2(nib(e, e20, m + 1), nib(o, o20, m + 1)), acc1);
-    }
+    for (int m = 0; m < 8; ++m) acc = __ffma2_rn(c[m], make_float2(nib(e, e20, m), nib(o, o20, m)), acc);
   } else {  // a = 2-bit plane word
     const uint32_t a22 = a >> 22;
 #pragma unroll
-    for (int p = 0; p < 8; p += 2) {
-      acc0 = __ffma2_rn(c[p], make_float2(fld2(a, a22, 2 * p), fld2(a, a22, 2 * p + 1)), acc0);
-      acc1 = __ffma2_rn(c[p + 1], make_float2(fld2(a, a22, 2 * p + 2), fld2(a, a22, 2 * p + 3)), acc1);
-    }
+    for (int p = 0; p < 8; ++p) acc = __ffma2_rn(c[p], make_float2(fld2(a, a22, 2 * p), fld2(a, a22, 2 * p + 1)), acc);
   }
-  return __fadd2_rn(acc0, acc1);
+  return acc;
 }
 
 // Two-way integer dot products (unsigned): d = c + a.lo16 * b.byte0 + a.hi16 * b.byte1
@@ -137,6 +131,12 @@ __device__ __forceinline__ void column_dot(uint32_t* acc, uint32_t w, uint32_t a
   acc[1] = dp2a_hi(a23, x1, dp2a_lo(a01, x1, acc[1]));
   acc[2] = dp2a_hi(a23, x2, dp2a_lo(a01, x2, acc[2]));
   acc[3] = dp2a_hi(a23, x3, dp2a_lo(a01, x3, acc[3]));
+}
+// Largest value over the warp (one instruction; NaN inputs are ignored).
+__device__ __forceinline__ float warp_max_f32(float x) {
+  float m;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(x));
+  return m;
 }
 // Round a non-negative float below 2^22 to the nearest integer in the low
 // bits of the result (added to 1.5 * 2^23, whose unit in the last place is 1).
@@ -250,7 +250,7 @@ struct Cfg {
 //         red float[D] (the owner's slice sums of every split),
 //         cnts int32[8] (every split's selection count)
 struct Smem {
-  size_t rings, ring_bytes, bars, qconst, q2buf, logits, ids, masks, xchg, scal, total;
+  size_t rings, ring_bytes, bars, qconst, q2buf, logits, ids, masks, gmax, xchg, scal, total;
 };
 // Per-warp buffer of 512 B, used twice per group: the key coefficients (128
 // floats) while the keys are read, then the group's value weights
@@ -267,7 +267,8 @@ __host__ __device__ inline Smem smem_plan(int stage_bytes, int nsw, int cg, int 
   s.logits = s.q2buf + static_cast<size_t>(kWarpBufBytes) * kNW;
   s.ids = s.logits + (logits ? 128 * static_cast<size_t>(cg) : 0);  // two block ids per group
   s.masks = s.ids + (logits ? 8 * static_cast<size_t>(cg) : 0);     // selection word per group
-  s.xchg = s.masks + (logits ? 4 * static_cast<size_t>(cg) : 0);
+  s.gmax = s.masks + (logits ? 4 * static_cast<size_t>(cg) : 0);    // largest logit per group
+  s.xchg = s.gmax + (logits ? 4 * static_cast<size_t>(cg) : 0);
   s.xchg = (s.xchg + 15) & ~static_cast<size_t>(15);
   s.scal = s.xchg + 16 * 8 * kNW + 4 * static_cast<size_t>(d) + 32;  // CTA scalars, warp counts
   s.total = s.scal + 32;
@@ -313,7 +314,8 @@ __device__ __forceinline__ int q2_slot(int k, int v) { return v * 16 + ((k + v) 
 template <int KIND, int D, bool FULLV, bool TAIL>
 __device__ __forceinline__ void group_step(const uint8_t* st, const float* qconst, float* q2buf, uint8_t* vbuf,
                                            const float* qfr, const __nv_bfloat16* res, int tok0, int nn,
-                                           int lane, int r, int k, float* logits_g, WarpState<D>& ws) {
+                                           int lane, int r, int k, float* logits_g, float* gmax_g,
+                                           WarpState<D>& ws) {
   using C = Cfg<KIND, D, FULLV>;
   using R = typename C::R;
   constexpr int CH = C::kCH, CW = C::kCW, NWRD = C::kNWRD, TS = C::kTS, TPL = C::kTPL, HALF = C::kHalf;
@@ -337,15 +339,15 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
   // ---- keys -> logits (scaled by 2^-E)
   float part[TPL];
   if constexpr (C::kQuant && !TAIL) {
-    // cooperative key coefficients of this group: lane l owns channels
-    // 4l..4l+3 (contiguous meta, conflict-free), q2 = qs * scale, and its
-    // share of alpha = sum_c qf_c * min_c
+    // cooperative key coefficients of this group: lane (r, k) prepares
+    // channels CW*k + 4r .. +3 of its own quarter (contiguous meta), q2 =
+    // qs * scale, and its share of alpha_k = sum over the quarter of qf_c *
+    // min_c; the quarter's 32 coefficients are then read back by its lanes
     float alpha;
     {
-      constexpr int kLanesUsed = D / 4;
       float a4 = 0.f;
-      if (kLanesUsed == 32 || lane < kLanesUsed) {
-        const int c0 = 4 * lane;
+      if (4 * r < CW) {
+        const int c0 = CW * k + 4 * r;
         const uint4 mw = *reinterpret_cast<const uint4*>(st + ((c0 < D / 2) ? 0 : HALF) + R::kKMetaOff +
                                                          (c0 % (D / 2)) * 4);
         const float4 qfv = *reinterpret_cast<const float4*>(qconst + c0);
@@ -355,17 +357,17 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
         float2 a2 = __fmul2_rn(make_float2(qfv.x, qfv.y), make_float2(bf16_hi(mw.x), bf16_hi(mw.y)));
         a2 = __ffma2_rn(make_float2(qfv.z, qfv.w), make_float2(bf16_hi(mw.z), bf16_hi(mw.w)), a2);
         a4 = a2.x + a2.y;
-        *reinterpret_cast<float4*>(q2buf + q2_slot<CW>(c0 / CW, (c0 % CW) / 4)) =
-            make_float4(q01.x, q01.y, q23.x, q23.y);
+        *reinterpret_cast<float4*>(q2buf + q2_slot<CW>(k, r)) = make_float4(q01.x, q01.y, q23.x, q23.y);
       }
+      // the quarter's lanes share lane % 4: sum over r
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a4 += __shfl_xor_sync(0xffffffffu, a4, o);
+      for (int o = 4; o < 32; o <<= 1) a4 += __shfl_xor_sync(0xffffffffu, a4, o);
       alpha = a4;
     }
     __syncwarp();
-    // each of the CH lanes of a token starts from alpha / CH (exact: CH is a
-    // power of two), so the all-reduce below adds alpha exactly once
-    alpha *= pow2i(-C::kE) / CH;
+    // every lane of a token row starts its partial logits from its quarter's
+    // alpha_k, so the transposed all-reduce over the row adds alpha once
+    alpha *= pow2i(-C::kE);
     float2 d[TPL];
 #pragma unroll
     for (int j = 0; j < TPL; ++j) d[j] = make_float2(alpha, 0.f);
@@ -452,9 +454,10 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
   __syncwarp();
 
   // ---- online softmax over the group (log2 units)
-  float gm = L;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+  const float gm = warp_max_f32(L);
+  if constexpr (C::kLogits) {
+    if (lane == 0) gmax_g[0] = gm;  // lets the selection pass skip groups far below tau
+  }
   if (gm > ws.m) {
     const float c = fast_exp2(ws.m - gm);  // 0 before the first group
     ws.l *= c;
@@ -467,7 +470,7 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
   // the group's own gap d below the running maximum (an integer, warp-
   // uniform): its weights are scaled by 2^d so that its largest is in (1/2, 1]
   const float dref = C::kQuant ? floorf(fminf(ws.m - gm, kMaxGroupGap)) : 0.f;
-  const float pw = pow2i(-static_cast<int>(dref));
+  const float pw = fast_exp2(-dref);  // an exact power of two: dref is an integer
   const float wg = valid ? fast_exp2(L - ws.m + dref) : 0.f;
   const float w = wg * pw;
   ws.l += w;
@@ -506,9 +509,7 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
     // fixed-point scale: every 2^d w * scale * sF stays below 2^15 (2^d w
     // <= 1); a larger scale than any seen so far lowers F for the whole warp
     if (__any_sync(0xffffffffu, smax >= ws.slim)) {
-      float x = smax;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+      const float x = warp_max_f32(smax);
       const int e = min(static_cast<int>((__float_as_uint(x * C::kMult) >> 23) & 0xFFu) - 127, kMaxFixedExp + 14);
       ws.F = min(14 - e, kMaxFixedExp);
       ws.sF = C::kMult * pow2i(ws.F);
@@ -606,6 +607,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   float* cacc = reinterpret_cast<float*>(smem + sp.rings + kCorrOff + D * 4);
   int32_t* ids_smem = reinterpret_cast<int32_t*>(smem + sp.ids);
   uint32_t* masks_smem = reinterpret_cast<uint32_t*>(smem + sp.masks);
+  float* gmax_smem = reinterpret_cast<float*>(smem + sp.gmax);
   float4* table = reinterpret_cast<float4*>(smem + sp.xchg);
   float* red = reinterpret_cast<float*>(smem + sp.xchg + 16 * 8 * kNW);
   int* cnts = reinterpret_cast<int*>(smem + sp.xchg + 16 * 8 * kNW + 4 * D);
@@ -791,9 +793,11 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       const uint8_t* st = ring + stage * STAGE;
       float* lg = logits + gi * kGroup;
       if (tok0 + kGroup <= nn)
-        group_step<KIND, D, FULLV, false>(st, qconst, q2buf, vbuf, qfr, res, tok0, nn, lane, r, k, lg, ws);
+        group_step<KIND, D, FULLV, false>(st, qconst, q2buf, vbuf, qfr, res, tok0, nn, lane, r, k, lg,
+                                            gmax_smem + gi, ws);
       else
-        group_step<KIND, D, FULLV, true>(st, qconst, q2buf, vbuf, qfr, res, tok0, nn, lane, r, k, lg, ws);
+        group_step<KIND, D, FULLV, true>(st, qconst, q2buf, vbuf, qfr, res, tok0, nn, lane, r, k, lg,
+                                           gmax_smem + gi, ws);
       // every shared-memory read of this stage has been consumed above, so
       // the stage can be refilled
       __syncwarp();
@@ -815,17 +819,29 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     const int col = lane % COLS, hb = lane / COLS, gv = (4 * col) / kGroup;
     float o[4];
     if constexpr (C::kQuant) {
-      // the value minima of the lane's group, summed over the owned tokens
-      float bsum[VG];
+      // the value minima of the lane's group gv, summed over every lane's
+      // owned tokens: a transposed all-reduce that halves the groups a lane
+      // keeps at each of the first log2(VG) steps (lane bit 4, then 3 picks
+      // the half, matching gv = lane / (32 / VG) for D = 128 and 64)
+      float bmine;
+      if constexpr (VG == 4) {
+        const bool up = lane & 16;
+        const float s0 = up ? ws.beta[0] : ws.beta[2], s1 = up ? ws.beta[1] : ws.beta[3];
+        const float q0 = (up ? ws.beta[2] : ws.beta[0]) + __shfl_xor_sync(0xffffffffu, s0, 16);
+        const float q1 = (up ? ws.beta[3] : ws.beta[1]) + __shfl_xor_sync(0xffffffffu, s1, 16);
+        const bool odd = lane & 8;
+        bmine = (odd ? q1 : q0) + __shfl_xor_sync(0xffffffffu, odd ? q0 : q1, 8);
 #pragma unroll
-      for (int g = 0; g < VG; ++g) {
-        bsum[g] = ws.beta[g];
+        for (int off = 4; off > 0; off >>= 1) bmine += __shfl_xor_sync(0xffffffffu, bmine, off);
+      } else {
+        static_assert(VG == 2, "value groups per token: 4 (D = 128) or 2 (D = 64)");
+        // D = 64: gv = col / 8 with col = lane % 16, i.e. lane bit 3
+        const bool odd = lane & 8;
+        bmine = (odd ? ws.beta[1] : ws.beta[0]) + __shfl_xor_sync(0xffffffffu, odd ? ws.beta[0] : ws.beta[1], 8);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) bsum[g] += __shfl_xor_sync(0xffffffffu, bsum[g], off);
+        for (int off = 16; off > 0; off >>= 1)
+          if (off != 8) bmine += __shfl_xor_sync(0xffffffffu, bmine, off);
       }
-      float bmine = bsum[0];
-#pragma unroll
-      for (int g = 1; g < VG; ++g) bmine = gv == g ? bsum[g] : bmine;
 #pragma unroll
       for (int f = 0; f < 4; ++f) o[f] = ws.facc[f];
       if constexpr (LPC == 2) {
@@ -927,7 +943,12 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       const bool valid = (g0 + gi) * kGroup + lane < nn;
       bool sel;
       if constexpr (C::kLogits) {
-        sel = valid && (fast_exp2(logits[gi * kGroup + lane] - m_g) * inv_z >= p.tau);
+        // a group whose largest weight is below tau selects nothing (the
+        // same fp32 test as the tokens', on its largest logit; warp-uniform)
+        if (fast_exp2(gmax_smem[gi] - m_g) * inv_z >= p.tau)
+          sel = valid && (fast_exp2(logits[gi * kGroup + lane] - m_g) * inv_z >= p.tau);
+        else
+          sel = false;
       } else {
         sel = C::kQ4 && valid;  // tau = 0: every token took its low plane in pass 1
       }
