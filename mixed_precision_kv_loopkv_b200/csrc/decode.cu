@@ -816,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     lw = ws.l;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
-    const int col = lane % COLS, hb = lane / COLS, gv = (4 * col) / kGroup;
+    const int col = lane % COLS, hb = lane / COLS;
     float o[4];
     if constexpr (C::kQuant) {
       // the value minima of the lane's group gv, summed over every lane's
