@@ -40,6 +40,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode-attention KV GB/s (% of B200 HBM peak) and µs per looped decode step"
+# what the decode kernel computes in: fp32 logits from the 2/4-bit key codes
+# (packed fp32 FMAs), values as u16 fixed-point weights x 2-bit codes (dp2a,
+# exact 32-bit integer group sums) accumulated in fp32
+DTYPE = "f32 logits; u16 weights x u2 codes (dp2a) values, f32 accumulate"
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -710,7 +714,7 @@ def main_arm(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": us_step / 1e3, "us_per_step": us_step,
             "pct_of_hbm_peak": value / world / peak * 100, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": cfg,
+            "vs_baseline": None, "dtype": DTYPE, "data": "synthetic", "config": cfg,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "kernel": "decode_kernel (all decode launches of one step, timed alone)",
