@@ -121,12 +121,11 @@ __device__ __forceinline__ uint32_t dp2a_hi(uint32_t a, uint32_t b, uint32_t c) 
 // acc[f] += the four tokens' codes of channel 4 col + f, weighted by the two
 // weight pairs a01 (tokens 0, 1 of the word) and a23 (tokens 2, 3).  Byte t
 // of w holds token t's channels 4 col .. 4 col + 3 at bits 0-1, 2-3, 4-5,
-// 6-7; fields 2 and 3 are read from w >> 4, so every field is isolated by one
-// AND and carries a factor 1 (f even) or 4 (f odd), undone at the end.
+// 6-7; field f is isolated in place by one AND and carries the factor 4^f
+// (a byte of at most 192), undone when the group's sums are added up.
 __device__ __forceinline__ void column_dot(uint32_t* acc, uint32_t w, uint32_t a01, uint32_t a23) {
-  const uint32_t y = w >> 4;
   const uint32_t x0 = w & 0x03030303u, x1 = w & 0x0C0C0C0Cu;
-  const uint32_t x2 = y & 0x03030303u, x3 = y & 0x0C0C0C0Cu;
+  const uint32_t x2 = w & 0x30303030u, x3 = w & 0xC0C0C0C0u;
   acc[0] = dp2a_hi(a23, x0, dp2a_lo(a01, x0, acc[0]));
   acc[1] = dp2a_hi(a23, x1, dp2a_lo(a01, x1, acc[1]));
   acc[2] = dp2a_hi(a23, x2, dp2a_lo(a01, x2, acc[2]));
@@ -137,11 +136,6 @@ __device__ __forceinline__ float warp_max_f32(float x) {
   float m;
   asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(x));
   return m;
-}
-// Round a non-negative float below 2^22 to the nearest integer in the low
-// bits of the result (added to 1.5 * 2^23, whose unit in the last place is 1).
-__device__ __forceinline__ uint32_t round_fixed(float w, float s) {
-  return __float_as_uint(fmaf(w, s, 12582912.f));
 }
 
 // Index of the sequence with rank r when the batch is ordered by decreasing
@@ -497,14 +491,20 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
     float sv[VG];
     float smax = 0.f;
 #pragma unroll
-    for (int g = 0; g < VG; ++g) {
-      const float sc = bf16_lo(mv[g]), mn = bf16_hi(mv[g]);
-      sv[g] = valid ? sc : 0.f;
-      smax = fmaxf(smax, sv[g]);
+    for (int g = 0; g < VG; g += 2) {
+      const float2 sc = make_float2(bf16_lo(mv[g]), bf16_lo(mv[g + 1]));
+      const float2 mn = make_float2(bf16_hi(mv[g]), bf16_hi(mv[g + 1]));
+      sv[g] = valid ? sc.x : 0.f;
+      sv[g + 1] = valid ? sc.y : 0.f;
+      smax = fmaxf(smax, fmaxf(sv[g], sv[g + 1]));
       // the minimum (plus the bucket midpoint of the high plane) of every
       // channel of the group, weighted once per token
-      const float base = C::kLogits ? fmaf(1.5f, sc, mn) : mn;
-      if (valid) ws.beta[g] = fmaf(w, base, ws.beta[g]);
+      const float2 base = C::kLogits ? __ffma2_rn(make_float2(1.5f, 1.5f), sc, mn) : mn;
+      if (valid) {
+        const float2 b = __ffma2_rn(make_float2(w, w), base, make_float2(ws.beta[g], ws.beta[g + 1]));
+        ws.beta[g] = b.x;
+        ws.beta[g + 1] = b.y;
+      }
     }
     // fixed-point scale: every 2^d w * scale * sF stays below 2^15 (2^d w
     // <= 1); a larger scale than any seen so far lowers F for the whole warp
@@ -517,14 +517,21 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
     }
     const float wF = wg * ws.sF;
     uint16_t* av = reinterpret_cast<uint16_t*>(vbuf);
+    const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23: round to an integer
 #pragma unroll
-    for (int g = 0; g < VG; ++g) {
-      av[g * 32 + tk] = static_cast<uint16_t>(round_fixed(wF, sv[g]));
-      if constexpr (C::kFourV) av[(VG + g) * 32 + tk] = static_cast<uint16_t>(round_fixed(0.25f * wF, sv[g]));
+    for (int g = 0; g < VG; g += 2) {
+      const float2 a = __ffma2_rn(make_float2(wF, wF), make_float2(sv[g], sv[g + 1]), magic);
+      av[g * 32 + tk] = static_cast<uint16_t>(__float_as_uint(a.x));
+      av[(g + 1) * 32 + tk] = static_cast<uint16_t>(__float_as_uint(a.y));
+      if constexpr (C::kFourV) {
+        const float2 b = __ffma2_rn(make_float2(0.25f * wF, 0.25f * wF), make_float2(sv[g], sv[g + 1]), magic);
+        av[(VG + g) * 32 + tk] = static_cast<uint16_t>(__float_as_uint(b.x));
+        av[(VG + g + 1) * 32 + tk] = static_cast<uint16_t>(__float_as_uint(b.y));
+      }
     }
     __syncwarp();
     // this lane's column: the weight pairs of its value group, token order;
-    // exact integer sums of the group (below 2^24), then added in fp32
+    // exact integer sums of the group (below 2^28), then added in fp32
     const uint32_t* ap = reinterpret_cast<const uint32_t*>(vbuf) + ((4 * col) / kGroup) * 16;
     uint32_t acc[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
@@ -555,10 +562,10 @@ __device__ __forceinline__ void group_step(const uint8_t* st, const float* qcons
         column_dot(acc, lw[3], l1.z, l1.w);
       }
     }
-    // back to value units: 2^-(F + d), and 1/4 for the odd fields
-    const float u0 = pow2i(-ws.F) * pw, u1 = 0.25f * u0;
+    // back to value units: 2^-(F + d), and 4^-f for field f
+    const float u0 = pow2i(-ws.F) * pw;
 #pragma unroll
-    for (int f = 0; f < 4; ++f) ws.facc[f] = fmaf(__uint2float_rn(acc[f]), (f & 1) ? u1 : u0, ws.facc[f]);
+    for (int f = 0; f < 4; ++f) ws.facc[f] = fmaf(__uint2float_rn(acc[f]), u0 * pow2i(-2 * f), ws.facc[f]);
   } else {
     float* wv = reinterpret_cast<float*>(vbuf);
     wv[tk] = w;
