@@ -19,7 +19,8 @@
 //     key meta, value high plane, value meta: 2048 B of the 2560-B 4-bit
 //     record at D = 128), completion on an mbarrier per stage;
 //   - the warp dequantises the keys at the cell's precision, forms the
-//     logits, keeps an online softmax and accumulates the high-plane values;
+//     logits, keeps an online softmax and accumulates the high-plane values
+//     (a reuse cell's optional current token joins as one exact token);
 //   - the splits exchange (max, sum) through distributed shared memory, so
 //     every CTA knows the exact normaliser Z before any low-plane read;
 //   - pass 2 re-reads the CTA's logits from shared memory, ballots the tokens
@@ -28,12 +29,18 @@
 //     the full 4-bit value);
 //   - a cluster-wide reduction over distributed shared memory writes bf16 out.
 //
-// Arithmetic for the HBM-bound inner loop (one FP32x2 FMA per two elements):
-// a code's bits are isolated in place with one AND and read as an fp32
+// Arithmetic of the inner loop.  Keys (one FP32x2 FMA per two codes): a
+// code's bits are isolated in place with one AND and read as an fp32
 // subnormal, code * 2^pos * 2^-149; the per-channel factor 2^(149 - pos - E)
-// is folded into the query (keys) or undone once per channel at the end
-// (values).  Subnormal FMA inputs are exact on this hardware (no FTZ), so
-// every product equals q * scale * code up to the global power of two 2^-E.
+// is folded into the query coefficient.  Subnormal FMA inputs are exact on
+// this hardware (no FTZ), so every product equals q * scale * code up to the
+// global power of two 2^-E, and the logits keep fp32 precision for the
+// selection.  Values (dp2a, two tokens per instruction): the value plane is
+// column-major within a block, so one word holds one 4-channel column of four
+// tokens; each token's softmax weight becomes 16-bit fixed-point weights
+// (one per 32-channel group, scaled to the group's own largest weight and the
+// largest value scale seen), each lane sums its column over the group's 32
+// tokens exactly in integers, and the sums are added in fp32.
 #include <float.h>
 #include <limits.h>
 
@@ -41,8 +48,6 @@
 #include <map>
 #include <mutex>
 #include <tuple>
-
-#include <cuda_fp16.h>
 
 #include "append_ops.cuh"
 #include "device_common.cuh"
