@@ -706,6 +706,10 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   const int nit = (!bad && cg > warp) ? (cg - warp + kNW - 1) / kNW : 0;
   const int g_unsafe = (nn - 1) / kGroup;  // may be written by the previous kernel
   const uint64_t pol = l2_evict_first_policy();
+  // record (block id, this KV head) lies at arena_h + id * rec_stride
+  const uint8_t* arena_h = p.arena + static_cast<size_t>(hk) * R::kBytes;
+  const size_t rec_stride = static_cast<size_t>(Hkv) * R::kBytes;
+  const uint32_t ring_addr = smem_addr(ring);
   const int32_t* btab = p.block_table + static_cast<size_t>(b) * p.max_blocks;
   // block ids of 16 iterations, two per iteration, spread over the lanes
   auto load_ids = [&](int it0, bool speculated) {
@@ -736,20 +740,18 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
     }
     const int id0 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base));
     const int id1 = __shfl_sync(0xffffffffu, ids, 2 * (it - ids_base) + 1);
-    if (C::kLogits && lane == 0) {  // kept for the low-plane gather of pass 2
-      ids_smem[2 * (warp + kNW * it)] = id0;
-      ids_smem[2 * (warp + kNW * it) + 1] = id1;
-    }
     if (lane == 0) {
+      if constexpr (C::kLogits) {  // kept for the low-plane gather of pass 2
+        ids_smem[2 * (warp + kNW * it)] = id0;
+        ids_smem[2 * (warp + kNW * it) + 1] = id1;
+      }
       const int stage = it % NSW;
       const uint32_t bar = bar0 + 8 * stage;
-      const uint32_t dst = smem_addr(ring + stage * STAGE);
+      const uint32_t dst = ring_addr + stage * STAGE;
       const uint32_t bytes = (id0 >= 0 ? LOAD : 0) + (id1 >= 0 ? LOAD : 0);
       mbar_arrive_expect_tx(bar, bytes);
-      if (id0 >= 0)
-        bulk_load(dst, p.arena + (static_cast<size_t>(id0) * Hkv + hk) * R::kBytes, LOAD, bar, pol);
-      if (id1 >= 0)
-        bulk_load(dst + C::kHalf, p.arena + (static_cast<size_t>(id1) * Hkv + hk) * R::kBytes, LOAD, bar, pol);
+      if (id0 >= 0) bulk_load(dst, arena_h + static_cast<size_t>(id0) * rec_stride, LOAD, bar, pol);
+      if (id1 >= 0) bulk_load(dst + C::kHalf, arena_h + static_cast<size_t>(id1) * rec_stride, LOAD, bar, pol);
     }
   };
 
@@ -947,7 +949,9 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   const float inv_z = live ? 1.f / z : 0.f;
 
   // ---- pass 2a: low-plane selection of every group of this warp
-  const bool want_mask = p.sel_mask != nullptr || p.sel_count != nullptr;
+  // only a 4-bit cell can select (its count); other kinds write their
+  // empty selection words only when asked for them
+  const bool want_mask = p.sel_mask != nullptr || (C::kQ4 && p.sel_count != nullptr);
   const bool gather = C::kLogits && p.tau < INFINITY;
   int cnt = 0;
   if (live && (gather || want_mask)) {
