@@ -15,7 +15,9 @@ C ABI, against the CPU oracle at |gpu - oracle| <= 2e-3 + 1e-2 |oracle|):
     sums land in the fp32 accumulators);
   * the exact current token of a reuse cell's own loop (k_cur, v_cur);
   * two host threads decoding the same kernel build with different shared
-    memory sizes at once.
+    memory sizes at once;
+  * the empty selection of the kinds that cannot select (2-bit, bf16, 4-bit
+    at tau = inf): zero words and counts written over buffers of ones.
 """
 
 import math
@@ -168,3 +170,30 @@ def test_two_threads_different_lengths():
         t.join()
     assert not errors, errors
     assert not bad
+
+
+@pytest.mark.parametrize("kind,tau", [("q2", 0.01), ("bf16", 0.01), ("q4", math.inf)])
+@pytest.mark.parametrize("with_mask", [True, False])
+def test_empty_selection_is_written(kind, tau, with_mask):
+    """Kinds that cannot select (2-bit, bf16) and a 4-bit cell at tau = inf
+    write zero selection words for every group of each sequence and a zero
+    count, over buffers that start out filled with ones (and a count alone,
+    without words, is still written)."""
+    from mixed_precision_kv_loopkv_b200 import loopkv_decode_attention
+    lens = [1, 31, 700, 3000]
+    k, v = _kv(len(lens), max(lens), 2, 128, seed=56)
+    kv, table, lens_d = store_tensors(kind, k, v, lens)
+    q = _q(len(lens), 2, 128, 57, 8.0)
+    sm, sc = mask_buffers(kv, len(lens))
+    sm.fill_(-1)
+    sc.fill_(-1)
+    out = loopkv_decode_attention(kv, 0, 0, q, table, lens_d, tau, 1.0, sel_mask=sm if with_mask else None,
+                                  sel_count=sc)
+    torch.cuda.synchronize()
+    assert torch.all(sc == 0)
+    if with_mask:
+        for b, n in enumerate(lens):
+            assert torch.all(sm[b, :, : (n + 31) // 32] == 0)
+            assert torch.all(sm[b, :, (n + 31) // 32:] == -1)   # words past the sequence are not touched
+    check_cell(kv, [kind], 0, {0: (k, v)}, q, table, lens_d, tau, 1.0,
+               [(b, h) for b in range(len(lens)) for h in range(2)], out=out)
