@@ -243,3 +243,26 @@ def test_maximum_context(kind):
     assert int(err) == 0
     check_cell(kv, [kind], 0, {0: (k, v)}, q, table_d, start + 1, 0.01, 1.0, [(0, 0), (0, 1), (1, 0)],
                out=out, sel_mask=sm, sel_count=sc)
+
+
+@pytest.mark.parametrize("B", [48, 64, 70])
+def test_ragged_batch_order(B):
+    """Batches are dispatched longest first (a rank of each sequence by
+    length, ties by index, over up to 64 sequences: both halves of a warp's
+    ranking for 33..64; beyond 64 the identity order): every sequence of a
+    ragged batch with repeated lengths is decoded exactly once, into its own
+    output row."""
+    from loopkv_testlib import seeded_bf16, store_tensors
+    rng = np.random.default_rng(B)
+    lens = rng.integers(1, 200, size=B)
+    lens[::7] = 96                                # ties
+    k = seeded_bf16((B, int(lens.max()), 2, 64), 60)
+    v = seeded_bf16((B, int(lens.max()), 2, 64), 61)
+    kv, table, lens_d = store_tensors("q4", k, v, lens.tolist())
+    q = seeded_bf16((B, 2, 64), 62, 0.5)
+    from mixed_precision_kv_loopkv_b200 import loopkv_decode_attention
+    sm, sc = mask_buffers(kv, B)
+    out = loopkv_decode_attention(kv, 0, 0, q, table, lens_d, 0.01, 1.0, sel_mask=sm, sel_count=sc)
+    torch.cuda.synchronize()
+    check_cell(kv, ["q4"], 0, {0: (k, v)}, q, table, lens_d, 0.01, 1.0,
+               [(b, h) for b in range(B) for h in range(2)], out=out, sel_mask=sm, sel_count=sc)
