@@ -17,7 +17,9 @@ C ABI, against the CPU oracle at |gpu - oracle| <= 2e-3 + 1e-2 |oracle|):
   * two host threads decoding the same kernel build with different shared
     memory sizes at once;
   * the empty selection of the kinds that cannot select (2-bit, bf16, 4-bit
-    at tau = inf): zero words and counts written over buffers of ones.
+    at tau = inf): zero words and counts written over buffers of ones;
+  * a dense selection (tau = 1e-6 on flat attention: nearly every token
+    gathers its low plane in pass 2).
 """
 
 import math
@@ -197,3 +199,22 @@ def test_empty_selection_is_written(kind, tau, with_mask):
             assert torch.all(sm[b, :, (n + 31) // 32:] == -1)   # words past the sequence are not touched
     check_cell(kv, [kind], 0, {0: (k, v)}, q, table, lens_d, tau, 1.0,
                [(b, h) for b in range(len(lens)) for h in range(2)], out=out)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_dense_selection(d):
+    """tau = 1e-6 on flat attention selects nearly every token: the gather of
+    pass 2 then walks every group of every warp, four rows per round trip;
+    the output matches the oracle and, within the tolerance, the uniform
+    4-bit result (tau = 0)."""
+    lens = [1, 33, 700, 2000]
+    k, v = _kv(len(lens), max(lens), 2, d, seed=58)
+    kv, table, lens_d = store_tensors("q4", k, v, lens)
+    q = _q(len(lens), 2, d, 59, 0.5)
+    pairs = [(b, h) for b in range(len(lens)) for h in range(2)]
+    out, sm, sc = _decode(kv, q, table, lens_d, 1e-6)
+    check_cell(kv, ["q4"], 0, {0: (k, v)}, q, table, lens_d, 1e-6, 1.0, pairs, out=out, sel_mask=sm,
+               sel_count=sc)
+    assert int(sc.sum()) > 0.99 * 2 * sum(lens)
+    full, _, _ = _decode(kv, q, table, lens_d, 0.0)
+    assert torch.allclose(out.float(), full.float(), rtol=1e-2, atol=ATOL)
