@@ -894,6 +894,11 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
 
   const int HC = head_cl ? 1 << p.g_log2 : 1;
   const int rbase = S * (h & (HC - 1));  // cluster rank of this head's split 0
+  // Kinds that cannot select (2-bit, bf16) need no normaliser before the
+  // combine: their splits meet once, each pushing its table entries and its
+  // channel sums in its own scale, and the owners rescale after that barrier.
+  constexpr bool kOneMeet = CLUSTER && !C::kQ4;
+  const int per_rank = D / S;
 
   // ---- publish (max, sum, error bits) of this warp into every split's table
   if constexpr (CLUSTER) cluster_wait();  // every CTA of the cluster has started
@@ -906,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       table[e] = ent;
     }
   }
-  if constexpr (CLUSTER) cluster_arrive_release();
+  if constexpr (CLUSTER && !kOneMeet) cluster_arrive_release();
 
   // ---- while the splits meet: this CTA's share of every channel in its own
   //      scale 2^-m_c (the warps' sub-group sums, rescaled and added)
@@ -922,7 +927,12 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       if (mw != -INFINITY) v = fmaf(fast_exp2(mw - m_c), wres_of(w)[c], v);
     }
     cacc[c] = v;
+    if constexpr (kOneMeet) {
+      // the owner of channel c gets it in this CTA's scale (m_c, from the table)
+      st_peer_f32(peer_addr(smem_addr(red + split * per_rank + c % per_rank), rbase + c / per_rank), v);
+    }
   }
+  if constexpr (kOneMeet) cluster_arrive_release();  // tables and sums are in place after the wait
   if constexpr (CLUSTER) cluster_wait_acquire(); else __syncthreads();
 
   // ---- global (max, normaliser, errors) from the local table
@@ -1098,9 +1108,30 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   if (lane == 0) cta_i[kSlotCnt0 + warp] = cnt;
   __syncthreads();  // every warp's sums, corrections and counts are in shared memory
 
+  if constexpr (kOneMeet) {
+    // ---- the owner's channels: every split's sum in the final units, added
+    //      in split order (the same arithmetic as the two-barrier combine)
+    if (threadIdx.x < per_rank) {
+      float v = 0.f;
+      for (int s = 0; s < S; ++s) {
+        float m_s = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) m_s = fmaxf(m_s, table[s * kNW + w].x);
+        float vs = 0.f;
+        if (live && m_s != -INFINITY) vs = red[s * per_rank + threadIdx.x] * fast_exp2(m_s - m_g) * inv_z;
+        v += vs;
+      }
+      p.out[(static_cast<size_t>(b) * p.H + h) * D + split * per_rank + threadIdx.x] = __float2bfloat16_rn(v);
+    }
+    if (split == 0 && threadIdx.x == 0) {
+      if (p.sel_count) p.sel_count[static_cast<size_t>(b) * p.H + h] = 0;
+      if (any_bad) flag_error(p.err, any_bad);
+    }
+    return;
+  }
+
   // ---- push this CTA's share of every channel, in the final units, to the
   //      split that owns the channel: rank s owns [s*D/S, (s+1)*D/S)
-  const int per_rank = D / S;
   if (threadIdx.x < D) {
     const int c = threadIdx.x;
     float v = 0.f;
