@@ -27,7 +27,9 @@
 //     with p >= tau and gathers only their 32-byte low-plane rows, adding
 //     p * scale * (lo - 1.5) per channel (turning the bucket midpoint into
 //     the full 4-bit value);
-//   - a cluster-wide reduction over distributed shared memory writes bf16 out.
+//   - a cluster-wide reduction over distributed shared memory writes bf16 out
+//     (kinds that cannot select push their sums with their (max, sum) table
+//     entries and meet once: the owners rescale after that one barrier).
 //
 // Arithmetic of the inner loop.  Keys (one FP32x2 FMA per two codes): a
 // code's bits are isolated in place with one AND and read as an fp32
