@@ -90,13 +90,18 @@ def test_ragged_lengths(kind, d, tau):
             assert int(sc[2, 0]) == 31
 
 
+@pytest.mark.parametrize("kind", ["q4", "q2", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("splits", [1, 2, 4, 8])
-def test_explicit_splits(splits):
-    w, kv, data, table, lens = _store_ragged("q4", 128, [7, 255, 777, 2048], heads=3, seed=3,
+def test_explicit_splits(kind, d, splits):
+    """Every split count of a cluster (a 4-bit cell's two-barrier combine, and
+    the single-barrier combine of 2-bit and bf16 cells, where each owner
+    rescales every split's channel sums), D 64 and 128."""
+    w, kv, data, table, lens = _store_ragged(kind, d, [7, 255, 777, 2048], heads=3, seed=3,
                                              splits=splits)
     q = query_for(w, 0, temperature=4.0)
     out, sm, sc = _decode(kv, 0, q, table, lens, 0.01)
-    check_cell(kv, ["q4"], 0, data, q, table, lens, 0.01, 1.0,
+    check_cell(kv, [kind], 0, data, q, table, lens, 0.01, 1.0,
                [(b, h) for b in range(4) for h in range(3)], out=out, sel_mask=sm, sel_count=sc)
 
 
@@ -116,6 +121,24 @@ def test_reuse_equals_source_with_own_query():
         assert torch.equal(out_r, out_s)
         check_cell(kv, plan, cell, data, q, table, lens, w.tau, 1.0,
                    [(0, h) for h in range(w.num_heads)], out=out_r, sel_mask=sm_r, sel_count=sc_r)
+
+
+@pytest.mark.parametrize("kind", ["q4", "q2", "bf16"])
+def test_bad_block_in_one_split_zeroes_the_whole_row(kind):
+    """A bad block id in one split of four: every split's owner learns of it
+    through the exchanged tables (both combines), the sequence-head's whole
+    output row is zero and the error bit is set; the other sequence is
+    unaffected."""
+    from mixed_precision_kv_loopkv_b200 import LOOPKV_DEVERR_BLOCK_ID
+    w, kv, data, table, lens = _store_ragged(kind, 128, [2048, 2048], heads=2, splits=4)
+    bad = table.clone()
+    bad[1, 70] = kv.num_blocks + 3          # block 70 of 128: the third split's chunk
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q = query_for(w, 0)
+    out, _, _ = _decode(kv, 0, q, bad, lens, 0.01, err=err)
+    assert int(err) & LOOPKV_DEVERR_BLOCK_ID
+    assert not out[1].any()
+    check_cell(kv, [kind], 0, data, q, table, lens, 0.01, 1.0, [(0, 0), (0, 1)], out=out)
 
 
 def test_bad_block_id_and_length_are_flagged():
