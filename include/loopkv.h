@@ -211,6 +211,8 @@ LOOPKV_API loopkv_status loopkv_quantize_append(const loopkv_config* cfg, const 
  *                 * block_size / 32); bit t%32 of word t/32 = token t took its low
  *                 plane; words past ceil(seq_len/32) are not written
  *   sel_count   : optional device int32 [batch][H], number of selected tokens
+ *                 (2-bit and bf16 sources have no low plane: zero words, zero
+ *                 counts)
  *   err_flag    : optional device int32
  * Errors: INVALID_ARG for tau < 0 or NaN, null required pointers, only one of
  * k_cur / v_cur, batch outside [0, max_batch]; BAD_PLAN; UNSUPPORTED for
