@@ -967,16 +967,12 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
   const bool gather = C::kLogits && p.tau < INFINITY;
   int cnt = 0;
   if (live && (gather || want_mask)) {
-    for (int gi = warp; gi < cg; gi += kNW) {
+    // the selection word of group gi (all lanes call; warp-uniform gi)
+    auto select_group = [&](int gi) {
       const bool valid = (g0 + gi) * kGroup + lane < nn;
       bool sel;
       if constexpr (C::kLogits) {
-        // a group whose largest weight is below tau selects nothing (the
-        // same fp32 test as the tokens', on its largest logit; warp-uniform)
-        if (fast_exp2(gmax_smem[gi] - m_g) * inv_z >= p.tau)
-          sel = valid && (fast_exp2(logits[gi * kGroup + lane] - m_g) * inv_z >= p.tau);
-        else
-          sel = false;
+        sel = valid && (fast_exp2(logits[gi * kGroup + lane] - m_g) * inv_z >= p.tau);
       } else {
         sel = C::kQ4 && valid;  // tau = 0: every token took its low plane in pass 1
       }
@@ -994,13 +990,35 @@ __global__ void __launch_bounds__(kThreads, MINB) decode_kernel(const DecodePara
       if (HC > 1) {
         // into the same split of every head of the group (itself included)
         if (lane < HC && mask) or_peer_u32(peer_addr(smem_addr(masks_smem + gi), split + S * lane), mask);
-        continue;
+        return;
       }
       if (lane == 0) {
         if (p.sel_mask) p.sel_mask[(static_cast<size_t>(b) * p.H + h) * p.mask_words + g0 + gi] = mask;
         if constexpr (C::kLogits) masks_smem[gi] = mask;
       }
       cnt += __popc(mask);
+    };
+    if constexpr (C::kLogits) {
+      // a group whose largest weight is below tau selects nothing (the same
+      // fp32 test as the tokens', on its largest logit): 32 groups tested at
+      // once, one per lane, and only the groups that pass are walked
+      const int ngw = cg > warp ? (cg - warp + kNW - 1) / kNW : 0;
+      for (int base = 0; base < ngw; base += 32) {
+        const int gl = warp + kNW * (base + lane);
+        const bool pass = base + lane < ngw && fast_exp2(gmax_smem[gl] - m_g) * inv_z >= p.tau;
+        if (base + lane < ngw && !pass && HC == 1) {
+          if (p.sel_mask) p.sel_mask[(static_cast<size_t>(b) * p.H + h) * p.mask_words + g0 + gl] = 0u;
+          masks_smem[gl] = 0u;
+        }
+        uint32_t todo = __ballot_sync(0xffffffffu, pass);
+        while (todo) {
+          const int j = __ffs(todo) - 1;
+          todo &= todo - 1u;
+          select_group(warp + kNW * (base + j));
+        }
+      }
+    } else {
+      for (int gi = warp; gi < cg; gi += kNW) select_group(gi);
     }
   }
   if (C::kLogits && HC > 1) {
